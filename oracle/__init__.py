@@ -1,0 +1,39 @@
+"""Oracle: a plain, slow, float64 CPU statement of one block-wise FIFO denoising
+queue, used ONLY as test infrastructure.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this package.  The product path (the CUDA library and
+its Python binding) never imports, links or executes anything here, and this
+package never imports the product.  The two share only the seeded input
+generator in ``synth`` (which holds none of the method's arithmetic).
+
+Source of the method: the DualParal write-up
+"双重并行：让AI视频生成突破时长限制，新加坡国立大学团队实现分钟级长视频创作"
+(techwalker.com, 2025-05-30), on "Minute-Long Videos with Dual Parallelisms":
+
+* §一 (dual-parallel architecture): the video is cut into non-overlapping
+  temporal chunks, each at its own noise level, later chunks noisier; one
+  inference step denoises all chunks at once.
+* §二 (FIFO queue and block-wise denoising): queue elements are chunks that
+  share one noise level, decreasing from T at the tail to 1 at the head; after
+  every diffusion step each chunk moves one place forward, a fresh noisy chunk
+  enters at the tail and the clean one leaves at the head for decoding.
+* §三 (feature cache and coordinated noise init): a chunk needs its neighbour's
+  information only in self-attention; the neighbour's self-attention K/V are
+  reused from a cache instead of concatenating the neighbour's input;
+  cross-attention and the FFN are strictly per chunk.
+
+The pages give no formula for the DiT block, the timestep embedding or the
+flow parameterisation.  Every step they leave open is written here in its
+plainest form and marked ``reading:`` at the point of use.
+
+Parity status: the self-attention, softmax, layer norm, modulation, GELU, SiLU,
+sinusoid, patch (un)folding, Euler update and queue bookkeeping are pinned by
+tests that do not reuse this code (closed forms, brute-force loops, textbook
+values, invariants and a hand-derived queue trace).  The composition of these
+pieces into the full DiT velocity has no printed value on the pages to pin it
+against: "parity unpinned" for ``dit.velocity`` beyond the invariants the tests
+check (gates, causality of the predecessor link, batch independence).
+"""
+
+from . import dit, fifo  # noqa: F401
