@@ -1,0 +1,348 @@
+// Persistent tcgen05 GEMM for sm_100a: C = A[M][K] . W[N][K]^T with the fused
+// epilogues of the DiT block (bias; bias+GELU; gated or plain residual add into
+// the fp32 stream; bias + copy of the neighbour-cache columns; the head's
+// Euler scatter into the latent ring).
+//
+// Layout: 128 x BN output tiles, K in blocks of 64 (one 128-byte swizzled row
+// per operand row).  One CTA per SM, 6 warps:
+//   warp 0      TMA producer (one thread): A and W tiles into a STAGES-deep ring
+//   warp 1      TMEM owner + MMA issuer (one thread): 4 x tcgen05.mma
+//               (M=128, N=BN, K=16) per k-block into one of two TMEM accumulators
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (thread = row),
+//               fused epilogue, 16-byte stores; frees the accumulator so the
+//               next tile's MMAs overlap this tile's epilogue.
+// Tiles are walked row-block-major so the CTAs in flight share A row blocks
+// through L2 while W stays L2-resident.  Every mbarrier wait is bounded.
+#include <mutex>
+
+#include "tc_common.cuh"
+
+namespace dp {
+
+using namespace tc;
+
+namespace {
+
+constexpr int BM = 128, BK = 64;
+
+__device__ __forceinline__ void store_bf16x32(bf16* dst, const float (&v)[32]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      __nv_bfloat162 p = __floats2bfloat162_rn(v[8 * i + 2 * j], v[8 * i + 2 * j + 1]);
+      w[j] = *reinterpret_cast<uint32_t*>(&p);
+    }
+    d4[i] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// Fused epilogue for 32 consecutive columns [col0, col0+32) of one row.
+__device__ __forceinline__ void epilogue32(const EpiParams& e, int row, int col0, float (&v)[32]) {
+  if (e.bias) {
+    const float4* b4 = reinterpret_cast<const float4*>(e.bias + col0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float4 b = b4[i];
+      v[4 * i] += b.x;
+      v[4 * i + 1] += b.y;
+      v[4 * i + 2] += b.z;
+      v[4 * i + 3] += b.w;
+    }
+  }
+  switch (e.mode) {
+    case EPI_GELU:
+#pragma unroll
+      for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
+      store_bf16x32((bf16*)e.out + (long long)row * e.ldo + col0, v);
+      break;
+    case EPI_STORE:
+      if (e.out_f32) {
+        float4* o = reinterpret_cast<float4*>((float*)e.out + (long long)row * e.ldo + col0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      } else {
+        store_bf16x32((bf16*)e.out + (long long)row * e.ldo + col0, v);
+        if (e.cache && row >= e.cache_row0 && row < e.cache_row0 + e.cache_rows &&
+            col0 >= e.cache_col0)
+          store_bf16x32((bf16*)e.cache + (long long)(row - e.cache_row0) * e.ldc + (col0 - e.cache_col0), v);
+      }
+      break;
+    case EPI_RESID:
+    case EPI_RESID_GATED: {
+      float4* x = reinterpret_cast<float4*>(e.resid + (long long)row * e.ldr + col0);
+      const float4* g = nullptr;
+      if (e.mode == EPI_RESID_GATED) {
+        const int c = row / e.rows_per_chunk;
+        const long long sel = e.chunk_sel ? e.chunk_sel[c] : c;
+        g = reinterpret_cast<const float4*>(e.gate + sel * e.gate_stride + col0);
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float4 r = x[i];
+        if (g) {
+          const float4 gg = g[i];
+          r.x = fmaf(gg.x, v[4 * i], r.x);
+          r.y = fmaf(gg.y, v[4 * i + 1], r.y);
+          r.z = fmaf(gg.z, v[4 * i + 2], r.z);
+          r.w = fmaf(gg.w, v[4 * i + 3], r.w);
+        } else {
+          r.x += v[4 * i];
+          r.y += v[4 * i + 1];
+          r.z += v[4 * i + 2];
+          r.w += v[4 * i + 3];
+        }
+        x[i] = r;
+      }
+      break;
+    }
+    case EPI_EULER: {
+      const float ds = e.dsig[row / e.rows_per_chunk];
+#pragma unroll 4
+      for (int i = 0; i < 32; ++i) e.ring[euler_index(e, row, col0 + i, e.rows_per_chunk)] += ds * v[i];
+      break;
+    }
+    default:
+      break;
+  }
+}
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const unsigned long long t0 = globaltimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer() - t0 > kWaitLimitNs) return;
+  }
+}
+
+template <int BN, int STAGES>
+__global__ void __launch_bounds__(192, 1)
+gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+               int M, int N, int K, EpiParams e, int* status) {
+  constexpr uint32_t A_BYTES = BM * BK * 2;
+  constexpr uint32_t B_BYTES = BN * BK * 2;
+  constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr uint32_t TMEM_COLS = 2 * BN;
+  constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, 0, 0);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ uint64_t full_bar[STAGES], empty_bar[STAGES], tfull_bar[2], tempty_bar[2], done_bar;
+  __shared__ uint32_t tmem_base_sh;
+  __shared__ volatile int abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tiles_n = (N + BN - 1) / BN;
+  const int tiles_m = (M + BM - 1) / BM;
+  const int num_tiles = tiles_n * tiles_m;
+  const int kblocks = K / BK;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < STAGES; ++i) {
+      mbar_init(&full_bar[i], 1);
+      mbar_init(&empty_bar[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&tfull_bar[i], 1);
+      mbar_init(&tempty_bar[i], 128);
+    }
+    mbar_init(&done_bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(&tmem_base_sh, TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA);
+    prefetch_tmap(&tmB);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tmem_base_sh;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, issued_par = 0;  // per-stage bit masks for the drain
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, ST_TIMEOUT_GEMM)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * STAGE_BYTES;
+          mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
+          tma_load_2d(sa, &tmA, kb * BK, m0, &full_bar[stage]);
+          tma_load_2d(sa + A_BYTES, &tmB, kb * BK, n0, &full_bar[stage]);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (abort_flag) {  // let copies in flight land before the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+          if (issued & (1u << s)) drain_wait(&full_bar[s], (issued_par >> s) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++it) {
+        const int buf = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(&tempty_bar[buf], acc_phase ^ 1, &abort_flag, status, ST_TIMEOUT_GEMM)) break;
+        tc_fence_after();
+        const uint32_t dtm = tmem_base + buf * BN;
+        for (int kb = 0; kb < kblocks; ++kb) {
+          if (!mbar_wait(&full_bar[stage], phase, &abort_flag, status, ST_TIMEOUT_GEMM)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+          const uint64_t ad = desc_sw128(sa, 16, 1024);
+          const uint64_t bd = desc_sw128(sa + A_BYTES, 16, 1024);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k)  // +32 bytes along K per step = +2 in the address field
+            mma_bf16_ss(dtm, ad + 2 * k, bd + 2 * k, IDESC, (kb | k) != 0);
+          mma_commit(&empty_bar[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (ok) mma_commit(&tfull_bar[buf]);
+      }
+      mma_commit(&done_bar);
+      drain_wait(&done_bar, 0);
+    }
+    __syncwarp();
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
+    const int rloc = quad * 32 + lane;
+    int it = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+      const int buf = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      if (!mbar_wait(&tfull_bar[buf], acc_phase, &abort_flag, status, ST_TIMEOUT_GEMM)) break;
+      tc_fence_after();
+      const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
+      const int row = m0 + rloc;
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + c * 32, v);
+        const int col0 = n0 + c * 32;
+        if (row < M && col0 < N) epilogue32(e, row, col0, v);
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty_bar[buf]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int sm_count() {
+  static int n = 0;
+  if (!n) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (n <= 0) n = 148;
+  }
+  return n;
+}
+
+}  // namespace
+
+// bf16 [rows][cols] row-major with row stride `ld` elements; box box_rows x 64.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, long long rows, long long cols, long long ld,
+                    int box_rows, int box_cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool gemm_tc_supported(long long lda, int M, int N, int K) {
+  return M > 0 && N > 0 && K > 0 && K % BK == 0 && N % 32 == 0 && lda % 8 == 0 && lda >= K;
+}
+
+template <int BN, int STAGES>
+static cudaError_t launch_tc(const bf16* A, long long lda, const bf16* W, int M, int N, int K,
+                             const EpiParams& e, int* status, cudaStream_t s) {
+  constexpr int SMEM = STAGES * (BM * BK * 2 + BN * BK * 2) + 1024;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  CUtensorMap ta, tb;
+  if (!make_tmap_bf16(&ta, A, M, K, lda, BM, BK)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16(&tb, W, N, K, K, BN, BK)) return cudaErrorInvalidValue;
+  const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
+  const int grid = tiles < sm_count() ? tiles : sm_count();
+  gemm_tc_kernel<BN, STAGES><<<grid, 192, SMEM, s>>>(ta, tb, M, N, K, e, status);
+  return cudaGetLastError();
+}
+
+cudaError_t gemm_tc(const bf16* A, long long lda, const bf16* W, int M, int N, int K,
+                    const EpiParams& e, int* status, cudaStream_t s) {
+  if (!gemm_tc_supported(lda, M, N, K)) return cudaErrorInvalidValue;
+  if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(W)) & 15) return cudaErrorInvalidValue;
+  if (N % 256 == 0) return launch_tc<256, 4>(A, lda, W, M, N, K, e, status, s);
+  if (N % 128 == 0) return launch_tc<128, 6>(A, lda, W, M, N, K, e, status, s);
+  return launch_tc<64, 8>(A, lda, W, M, N, K, e, status, s);
+}
+
+}  // namespace dp

@@ -1,0 +1,258 @@
+// Memory-bound kernels of the queue step: LayerNorm + adaLN modulation, the
+// patch gather from the latent ring, per-level timestep features, table
+// broadcast, the seeded noise generator and dtype conversions.
+#include "common.cuh"
+
+namespace dp {
+
+// ---------------------------------------------------------------------------
+// LayerNorm (no affine, biased variance, eps 1e-6) + adaLN shift/scale.
+// One 128-thread block per row, 128-bit loads of x; the row stays in
+// registers between the mean, variance and output passes (d <= 6144).
+// ---------------------------------------------------------------------------
+constexpr int LN_THREADS = 128;
+constexpr int LN_MAXV = 12;
+
+template <bool OUT_F32>
+__global__ void __launch_bounds__(LN_THREADS) ln_mod_kernel(LnParams p) {
+  __shared__ float red[LN_THREADS / 32];
+  const int row = blockIdx.x;
+  const int nv = p.d >> 2;
+  const float4* xr = reinterpret_cast<const float4*>(p.x + (long long)row * p.ldx);
+  float4 v[LN_MAXV];
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < LN_MAXV; ++i) {
+    const int idx = threadIdx.x + i * LN_THREADS;
+    if (idx < nv) {
+      v[i] = xr[idx];
+      s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+    }
+  }
+  const float mean = block_sum<LN_THREADS / 32>(s, red) / (float)p.d;
+  float ss = 0.0f;
+#pragma unroll
+  for (int i = 0; i < LN_MAXV; ++i) {
+    const int idx = threadIdx.x + i * LN_THREADS;
+    if (idx < nv) {
+      const float a = v[i].x - mean, b = v[i].y - mean, c = v[i].z - mean, d = v[i].w - mean;
+      ss += (a * a + b * b) + (c * c + d * d);
+    }
+  }
+  const float var = block_sum<LN_THREADS / 32>(ss, red) / (float)p.d;
+  const float rstd = 1.0f / sqrtf(var + 1e-6f);
+  const float4* sh = nullptr;
+  const float4* sc = nullptr;
+  if (p.shift) {
+    const int c = row / p.rows_per_chunk;
+    const long long sel = p.chunk_sel ? p.chunk_sel[c] : c;
+    sh = reinterpret_cast<const float4*>(p.shift + sel * p.mod_stride);
+    sc = reinterpret_cast<const float4*>(p.scale + sel * p.mod_stride);
+  }
+#pragma unroll
+  for (int i = 0; i < LN_MAXV; ++i) {
+    const int idx = threadIdx.x + i * LN_THREADS;
+    if (idx < nv) {
+      float4 o;
+      o.x = (v[i].x - mean) * rstd;
+      o.y = (v[i].y - mean) * rstd;
+      o.z = (v[i].z - mean) * rstd;
+      o.w = (v[i].w - mean) * rstd;
+      if (sh) {
+        const float4 a = sh[idx], b = sc[idx];
+        o.x = o.x * (1.0f + b.x) + a.x;
+        o.y = o.y * (1.0f + b.y) + a.y;
+        o.z = o.z * (1.0f + b.z) + a.z;
+        o.w = o.w * (1.0f + b.w) + a.w;
+      }
+      if (OUT_F32) {
+        reinterpret_cast<float4*>((float*)p.out + (long long)row * p.ldo)[idx] = o;
+      } else {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(o.z, o.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        reinterpret_cast<uint2*>((bf16*)p.out + (long long)row * p.ldo)[idx] = pk;
+      }
+    }
+  }
+}
+
+cudaError_t layernorm_mod(const LnParams& p, cudaStream_t s) {
+  if (p.M <= 0) return cudaSuccess;
+  if (p.out_f32) ln_mod_kernel<true><<<p.M, LN_THREADS, 0, s>>>(p);
+  else ln_mod_kernel<false><<<p.M, LN_THREADS, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Patch gather: ring slot [C][F][H][W] -> token rows [Lc][C*pt*ph*pw].
+// One thread per output element; consecutive threads walk the feature index.
+// ---------------------------------------------------------------------------
+template <typename TO>
+__global__ void gather_kernel(const float* __restrict__ ring, long long chunk_numel,
+                              const int* __restrict__ chunk_slot, long long total, int Lc,
+                              int C, int F, int H, int W, int pt, int ph, int pw, TO* out) {
+  const int P = C * pt * ph * pw;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long row = i / P;
+    const int col = (int)(i - row * P);
+    const int c = (int)(row / Lc), t = (int)(row - (long long)c * Lc);
+    const int hq = H / ph, wq = W / pw;
+    const int fq = t / (hq * wq), rem = t - fq * (hq * wq);
+    const int yq = rem / wq, xq = rem - yq * wq;
+    const int dx = col % pw, dy = (col / pw) % ph, dt = (col / (pw * ph)) % pt;
+    const int cc = col / (pw * ph * pt);
+    const long long lat = (((long long)cc * F + fq * pt + dt) * H + yq * ph + dy) * W + xq * pw + dx;
+    out[i] = from_f<TO>(ring[(long long)chunk_slot[c] * chunk_numel + lat]);
+  }
+}
+
+cudaError_t gather_patches(const float* ring, long long chunk_numel, const int* chunk_slot,
+                           int n_chunks, int C, int F, int H, int W, int pt, int ph, int pw,
+                           void* out, int out_f32, cudaStream_t s) {
+  const int Lc = (F / pt) * (H / ph) * (W / pw);
+  const long long total = (long long)n_chunks * Lc * C * pt * ph * pw;
+  if (total <= 0) return cudaSuccess;
+  const int threads = 256;
+  const long long blocks = (total + threads - 1) / threads;
+  const int grid = (int)(blocks < 148 * 32 ? blocks : 148 * 32);
+  if (out_f32)
+    gather_kernel<float><<<grid, threads, 0, s>>>(ring, chunk_numel, chunk_slot, total, Lc, C, F,
+                                                  H, W, pt, ph, pw, (float*)out);
+  else
+    gather_kernel<bf16><<<grid, threads, 0, s>>>(ring, chunk_numel, chunk_slot, total, Lc, C, F,
+                                                 H, W, pt, ph, pw, (bf16*)out);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Sinusoidal features of t_j = 1000 j / T, j = 1..T: [cos(t w_i), sin(t w_i)],
+// w_i = 10000^(-i/(D/2)).  Evaluated in double, rounded once to float.
+// ---------------------------------------------------------------------------
+__global__ void timestep_kernel(int T, int D, float* out) {
+  const int j = blockIdx.x + 1;
+  const int half = D / 2;
+  const double t = 1000.0 * ((double)j / (double)T);
+  for (int i = threadIdx.x; i < half; i += blockDim.x) {
+    const double w = pow(10000.0, -(double)i / (double)half);
+    out[(long long)(j - 1) * D + i] = (float)cos(t * w);
+    out[(long long)(j - 1) * D + half + i] = (float)sin(t * w);
+  }
+}
+
+cudaError_t timestep_features(int T, int D, float* out, cudaStream_t s) {
+  timestep_kernel<<<T, 128, 0, s>>>(T, D, out);
+  return cudaGetLastError();
+}
+
+__global__ void add_tables_kernel(const float* m, const float* table, int T, int L, int w,
+                                  float* out) {
+  const long long total = (long long)T * L * w;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int c = (int)(i % w);
+    const long long jl = i / w;
+    const int l = (int)(jl % L);
+    const int j = (int)(jl / L);
+    out[i] = m[(long long)j * w + c] + table[(long long)l * w + c];
+  }
+}
+
+cudaError_t add_layer_tables(const float* m, const float* table, int T, int L, int w,
+                             float* out, cudaStream_t s) {
+  add_tables_kernel<<<1024, 256, 0, s>>>(m, table, T, L, w, out);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Seeded N(0,1): SplitMix64 (Steele, Lea, Flood 2014) stream keyed by
+// (seed, a, b) and the Box-Muller transform (1958) in double, as in the
+// host-side generator.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ unsigned long long mix64(unsigned long long z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+__global__ void normal_kernel(unsigned long long key, float* out, long long n) {
+  const unsigned long long g = 0x9E3779B97F4A7C15ull;
+  const long long npairs = (n + 1) / 2;
+  for (long long p = blockIdx.x * (long long)blockDim.x + threadIdx.x; p < npairs;
+       p += (long long)gridDim.x * blockDim.x) {
+    const unsigned long long d0 = mix64(key + (unsigned long long)(2 * p + 1) * g) >> 11;
+    const unsigned long long d1 = mix64(key + (unsigned long long)(2 * p + 2) * g) >> 11;
+    const double u1 = ((double)d0 + 1.0) * 0x1.0p-53;
+    const double u2 = (double)d1 * 0x1.0p-53;
+    const double r = sqrt(-2.0 * log(u1));
+    const double th = 6.283185307179586476925 * u2;
+    out[2 * p] = (float)(r * cos(th));
+    if (2 * p + 1 < n) out[2 * p + 1] = (float)(r * sin(th));
+  }
+}
+
+static unsigned long long host_mix64(unsigned long long z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+
+cudaError_t normal_fill(unsigned long long seed, unsigned long long a, unsigned long long b,
+                        float* out, long long n, cudaStream_t s) {
+  const unsigned long long g = 0x9E3779B97F4A7C15ull;
+  unsigned long long k = host_mix64((seed + 1) * g);
+  k = host_mix64(k + (a + 1) * g);
+  k = host_mix64(k + (b + 1) * g);
+  normal_kernel<<<148 * 4, 256, 0, s>>>(k, out, n);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Conversions
+// ---------------------------------------------------------------------------
+__global__ void f32_to_bf16_kernel(const float* in, bf16* out, long long n) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x)
+    out[i] = __float2bfloat16_rn(in[i]);
+}
+__global__ void bf16_to_f32_kernel(const bf16* in, float* out, long long n) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x)
+    out[i] = __bfloat162float(in[i]);
+}
+
+cudaError_t convert_f32_to_bf16(const float* in, bf16* out, long long n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  f32_to_bf16_kernel<<<148 * 8, 256, 0, s>>>(in, out, n);
+  return cudaGetLastError();
+}
+cudaError_t convert_bf16_to_f32(const bf16* in, float* out, long long n, cudaStream_t s) {
+  if (n <= 0) return cudaSuccess;
+  bf16_to_f32_kernel<<<148 * 8, 256, 0, s>>>(in, out, n);
+  return cudaGetLastError();
+}
+
+__global__ void copy_rows_kernel(const void* in, int in_f32, long long ldi, void* out,
+                                 int out_f32, long long ldo, long long rows, long long cols) {
+  const long long total = rows * cols;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long r = i / cols, c = i - r * cols;
+    const float v = in_f32 ? ((const float*)in)[r * ldi + c]
+                           : __bfloat162float(((const bf16*)in)[r * ldi + c]);
+    if (out_f32) ((float*)out)[r * ldo + c] = v;
+    else ((bf16*)out)[r * ldo + c] = __float2bfloat16_rn(v);
+  }
+}
+
+cudaError_t copy_rows(const void* in, int in_f32, long long ldi, void* out, int out_f32,
+                      long long ldo, long long rows, long long cols, cudaStream_t s) {
+  if (rows * cols <= 0) return cudaSuccess;
+  copy_rows_kernel<<<148 * 8, 256, 0, s>>>(in, in_f32, ldi, out, out_f32, ldo, rows, cols);
+  return cudaGetLastError();
+}
+
+}  // namespace dp

@@ -1,0 +1,47 @@
+"""The C library loads and exports every entry point its headers declare (no GPU)."""
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+
+def declared_symbols():
+    names = set()
+    for h in ("dp.h", "dp_ops.h"):
+        src = open(os.path.join(ROOT, "include", h)).read()
+        names |= set(re.findall(r"^DP_API [^;(]*?\b(dp_\w+)\s*\(", src, flags=re.M))
+    return names
+
+
+def test_headers_declare_the_queue_abi():
+    names = declared_symbols()
+    for n in ("dp_model_create", "dp_queue_init", "dp_queue_step", "dp_queue_pop", "dp_destroy"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    from chunked_fifo_denoising_b200 import _binding as B
+    lib = B.lib()
+    names = declared_symbols()
+    for n in names:
+        assert hasattr(lib, n), n
+    assert names == set(B.EXPORTED), "binding and headers disagree"
+
+
+def test_param_numel_and_config_errors():
+    import ctypes as C
+    from chunked_fifo_denoising_b200 import _binding as B
+    import synth
+    m = synth.WORKLOADS["wan1.3b_480p"].model
+    cfg = B.dp_model_config(m.n_layers, m.dim, m.n_heads, m.ffn_dim, m.freq_dim, m.latent_ch,
+                            m.patch_t, m.patch_h, m.patch_w, m.text_len, m.text_in_dim, 0)
+    n = C.c_longlong()
+    for name, shape, per_layer in synth.param_specs(m):
+        assert B.dp_param_numel(cfg, B.PARAM_IDS[name], n) == 0
+        assert n.value == int(__import__("numpy").prod(shape)), name
+    bad = B.dp_model_config(*[getattr(cfg, f) for f, _ in cfg._fields_])
+    bad.n_heads = 7
+    assert B.dp_param_numel(bad, 0, n) == B.DP_ERR_INVALID_ARG
+    assert "n_heads" in B.dp_last_error() or "head" in B.dp_last_error()

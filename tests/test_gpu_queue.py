@@ -1,0 +1,240 @@
+"""Queue-level parity on the GPU through the C ABI (dp_queue_*), against the
+float64 oracle on identical seeded inputs:
+
+* fp32 validation mode, tiny workload: every popped chunk of the whole stream
+  within relative L2 1e-4;
+* bookkeeping (chunk ids, levels, positions, neighbour source, pop order)
+  exactly equal to the oracle queue on the (T, N) schedule of every workload;
+* bf16 production mode: one queue step from the same state within relative L2
+  2e-2 on the velocity of every chunk, on the persisted K/V and on the latents
+  (small workload; Wan-1.3B shapes with two layers);
+* error codes, the internal noise generator, flat device memory.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import synth  # noqa: E402
+from oracle import dit, fifo  # noqa: E402
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def rel_l2(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+def bf16_round(x):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).float().numpy()
+
+
+def make(w, precision, params=None, text=None, n_chunks=None, T=None, ready=2):
+    from chunked_fifo_denoising_b200 import Model, Queue
+    m, q = w.model, w.queue
+    params = synth.make_params(m) if params is None else params
+    text = synth.make_text(m) if text is None else text
+    model = Model(m, precision)
+    model.set_params(params)
+    queue = Queue(model, text, q.T if T is None else T, q.frames_per_chunk, q.lat_h, q.lat_w,
+                  q.n_chunks if n_chunks is None else n_chunks, ready_capacity=ready)
+    return model, queue, params, text
+
+
+def test_tiny_fp32_stream_matches_oracle():
+    w = synth.WORKLOADS["tiny_fp32"]
+    m, q = w.model, w.queue
+    model, queue, p, text = make(w, "fp32")
+    noise = [synth.make_noise(m, q, k) for k in range(q.n_chunks)]
+    fn = dit.make_velocity_fn(p, text, m, q.T)
+    ready, traces = fifo.run_stream(fn, lambda k: noise[k], q.T, q.n_chunks)
+    out = np.empty(q.chunk_shape(m), np.float32)
+    got = {}
+    for tr in traces:
+        info = queue.inspect()
+        assert info["step"] == tr.step
+        assert info["ids"] == tr.chunk_ids and info["levels"] == tr.levels
+        assert info["positions"] == tr.positions
+        assert info["head_pred"] == tr.head_pred
+        queue.step(noise[tr.step] if tr.step < q.n_chunks else None)
+        queue.sync()
+        popped = []
+        while True:
+            st, cid = queue.try_pop(out)
+            if st != 0:
+                break
+            popped.append(cid)
+            got[cid] = out.copy()
+        assert popped == tr.popped
+    assert queue.inspect()["drained"] == 1
+    assert list(got) == list(range(q.n_chunks))
+    for k, ref in ready:
+        assert rel_l2(got[k], ref) <= 1e-4, k
+    model.close()
+
+
+@pytest.mark.parametrize("name", list(synth.WORKLOADS))
+def test_bookkeeping_exact_on_every_schedule(name):
+    """The (T, N) schedule of each workload, run at full N on the tiny model."""
+    w = synth.WORKLOADS[name]
+    T, N = w.queue.T, w.queue.n_chunks
+    tiny = synth.WORKLOADS["tiny_fp32"]
+    model, queue, _, _ = make(tiny, "fp32", n_chunks=N, T=T)
+    _, traces = fifo.run_stream(lambda lat, lv, ids, kv, keep: ([np.zeros_like(x) for x in lat], None),
+                                lambda k: np.zeros((1, 1, 1, 1)), T, N)
+    assert len(traces) == N + T - 1
+    out = torch.empty(tiny.queue.chunk_shape(tiny.model), device="cuda")
+    order = []
+    for tr in traces:
+        info = queue.inspect()
+        assert (info["step"], info["ids"], info["levels"], info["positions"], info["head_pred"]) == \
+            (tr.step, tr.chunk_ids, tr.levels, tr.positions, tr.head_pred)
+        assert info["writes_cache"] == int(tr.levels[0] == 1)
+        assert info["slots"] == [k % (T + 2) for k in tr.chunk_ids]
+        queue.step(None)
+        while True:
+            st, cid = queue.try_pop(out)
+            if st != 0:
+                break
+            order.append(cid)
+    assert order == list(range(N))
+    assert queue.try_step(None) == 6  # DP_ERR_DRAINED
+    queue.sync()
+    model.close()
+
+
+def _one_step_parity(w, n_layers=None, seed_state=7):
+    """Queue state just before a step: chunks at levels 1, 2, 3 (no push), the
+    head's predecessor K/V persisted; compare one GPU step with the oracle."""
+    if n_layers is not None:
+        w = synth.truncated(w, n_layers)
+    m, q = w.model, w.queue
+    T = q.T
+    n_chunks = 20
+    step = n_chunks + T - 4          # chunks 17, 18, 19 at levels 1, 2, 3
+    head = n_chunks - 3
+    model, queue, p, text = make(w, "bf16", n_chunks=n_chunks)
+    rng = np.random.default_rng(seed_state)
+    lat = rng.standard_normal((3,) + q.chunk_shape(m)).astype(np.float32)
+    Lc = q.tokens_per_chunk(m)
+    kv = bf16_round(rng.standard_normal((m.n_layers, 2, Lc, m.dim)).astype(np.float32) * 0.5)
+    queue.load_state(step, n_chunks, lat, kv)
+    info = queue.inspect()
+    assert info["ids"] == [head, head + 1, head + 2] and info["levels"] == [1, 2, 3]
+    assert info["head_pred"] == 2 and info["writes_cache"] == 1
+    queue.step(None)
+    queue.sync()
+    popped = np.empty(q.chunk_shape(m), np.float32)
+    assert queue.pop(popped) == head
+    rest = queue.read_latents(2)
+    new_kv, kv_id = queue.read_pred_kv()
+    assert kv_id == head
+    # oracle
+    fn = dit.make_velocity_fn(p, text, m, T)
+    st = fifo.QueueState(T=T, n_chunks=n_chunks, step=step, next_id=n_chunks,
+                         entries=[fifo.Entry(head + i, 1 + i, lat[i].astype(np.float64)) for i in range(3)],
+                         pred_id=head - 1, pred_kv=[(kv[l, 0], kv[l, 1]) for l in range(m.n_layers)])
+    tr = fifo.queue_step(st, fn, None)
+    assert tr.popped == [head]
+    ref_pop = st.ready[0][1]
+    ref_rest = [e.latent for e in st.entries]
+    dsig = -1.0 / T
+    v_gpu = [(popped - lat[0]) / dsig] + [(rest[i] - lat[i + 1]) / dsig for i in range(2)]
+    v_ref = [(ref_pop - lat[0]) / dsig] + [(ref_rest[i] - lat[i + 1]) / dsig for i in range(2)]
+    errs = [rel_l2(a, b) for a, b in zip(v_gpu, v_ref)]
+    assert max(errs) <= 2e-2, errs
+    assert rel_l2(popped, ref_pop) <= 2e-2
+    for l in range(m.n_layers):
+        assert rel_l2(new_kv[l, 0], st.pred_kv[l][0]) <= 2e-2, l
+        assert rel_l2(new_kv[l, 1], st.pred_kv[l][1]) <= 2e-2, l
+    model.close()
+    return errs
+
+
+def test_bf16_step_small():
+    _one_step_parity(synth.WORKLOADS["small_bf16"])
+
+
+def test_bf16_step_wan13b_shapes_two_layers():
+    _one_step_parity(synth.WORKLOADS["wan1.3b_480p"], n_layers=2)
+
+
+def test_errors_full_empty_drained():
+    w = synth.WORKLOADS["tiny_fp32"]
+    model, queue, _, _ = make(w, "fp32", n_chunks=-1, T=2, ready=1)
+    out = np.empty(w.queue.chunk_shape(w.model), np.float32)
+    st, _ = queue.try_pop(out)
+    assert st == 4  # DP_ERR_EMPTY
+    queue.step(None)                      # chunk 0 at level 2
+    queue.step(None)                      # chunk 0 level 1 -> ready
+    assert queue.inspect()["n_ready"] == 1
+    queue.step(None)                      # uses the last free slot (T + 1 = 3 slots)
+    assert queue.try_step(None) == 5      # DP_ERR_FULL: chunk 0 and 1 wait for pop
+    assert queue.pop(out) == 0
+    queue.step(None)
+    queue.close_stream()
+    while queue.try_step(None) == 0:
+        pass
+    ids = []
+    while True:
+        st, cid = queue.try_pop(out)
+        if st != 0:
+            break
+        ids.append(cid)
+    assert ids == sorted(ids) and ids[0] == 1
+    assert queue.try_step(None) == 6
+    model.close()
+
+
+def test_internal_generator_matches_seeded_noise():
+    """NULL noise draws chunk k from the same SplitMix64/Box-Muller stream as
+    the host generator.  With the output layer at zero the step leaves it as is."""
+    w = synth.WORKLOADS["tiny_fp32"]
+    m, q = w.model, w.queue
+    p = synth.make_params(m)
+    p["out.w"] = np.zeros_like(p["out.w"])
+    p["out.b"] = np.zeros_like(p["out.b"])
+    model, queue, _, _ = make(w, "fp32", params=p)
+    queue.step(None)
+    queue.step(None)
+    lat = queue.read_latents(2)
+    for k in range(2):
+        ref = synth.make_noise(m, q, k)
+        assert np.allclose(lat[k], ref, rtol=1e-6, atol=1e-6)
+    model.close()
+
+
+def test_device_memory_flat_in_stream_length():
+    """Long-stream workload: memory after init is the same for 32, 64 and 128
+    chunks and the steps allocate nothing (two-layer model, zero weights)."""
+    from chunked_fifo_denoising_b200 import Model, Queue
+    w = synth.truncated(synth.WORKLOADS["wan1.3b_480p_long"], 2)
+    m, q = w.model, w.queue
+    model = Model(m, "bf16")
+    for name, shape, per_layer in synth.param_specs(m):
+        t = torch.zeros(shape, device="cuda")
+        model.set_params({name: [t] * m.n_layers if per_layer else t})
+    text = torch.zeros((m.text_len, m.text_in_dim), device="cuda")
+    torch.cuda.synchronize()
+    used = []
+    for n in (32, 64, 128):
+        free0 = torch.cuda.mem_get_info()[0]
+        queue = Queue(model, text, q.T, q.frames_per_chunk, q.lat_h, q.lat_w, n)
+        free1 = torch.cuda.mem_get_info()[0]
+        for _ in range(3):
+            queue.step(None)
+        queue.sync()
+        free2 = torch.cuda.mem_get_info()[0]
+        assert free2 == free1
+        used.append(free0 - free1)
+        queue.close()
+    assert used[0] == used[1] == used[2]
+    model.close()
