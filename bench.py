@@ -1,0 +1,339 @@
+"""Steady-state throughput of the FIFO denoising queue on B200 (one JSON line).
+
+A step is one dp_queue_step over a full queue (every level occupied: one
+batched DiT pass over all queued chunks, the Euler update in the ring, the
+push of a fresh N(0,1) chunk) plus the dp_queue_pop of the clean chunk.
+Workload: the Wan2.1-1.3B-shaped random-init model (30 layers, dim 1536,
+12 heads, FFN 8960), 480x832 video -> 16-ch 60x104 latent, chunks of 2 latent
+frames (3120 tokens), T = 50 levels, 512 prompt tokens.  Metric: latent
+frames/s (2 frames leave the queue per step) and the fraction of the bf16
+tensor-core peak reached by the step's algorithmic FLOPs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs N independent replicas (one queue per GPU, no collective on the
+data path), launched by torch.distributed.run.  --impl reference times the
+float64 CPU oracle on a bounded sample of the same step (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "latent frames/s per B200 (steady-state queue); % of bf16 tensor-core peak"
+UNIT = "latent frames/s"
+FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["_source"] = "measured"
+        return d
+    d = dict(FALLBACK)
+    d["_source"] = "fallback"
+    return d
+
+
+def step_flops(m, q, occ):
+    """Algorithmic FLOPs of one step with `occ` queued chunks, every chunk with
+    a full predecessor: per token per layer 12 d^2 + 4 d F + 4 (2 Lc) d + 4 Lt d,
+    plus the patch and head projections (2 * 64 * d each per token)."""
+    Lc = q.tokens_per_chunk(m)
+    d, F = m.dim, m.ffn_dim
+    per_tok_layer = 12 * d * d + 4 * d * F + 4 * (2 * Lc) * d + 4 * m.text_len * d
+    toks = occ * Lc
+    return toks * (m.n_layers * per_tok_layer + 2 * 2 * m.patch_dim * d)
+
+
+class Clocks:
+    """Samples nvidia-smi clocks and throttle reasons while alive."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = str(index)
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.Q,
+                                       "--format=csv,noheader,nounits", "-lms", "200"],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return None
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        sm, mx, reasons = [], 0.0, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.f.read().splitlines():
+            c = [x.strip() for x in ln.split(",")]
+            if len(c) < 9 or c[0] != self.index:
+                continue
+            try:
+                sm.append(float(c[1]))
+                mx = max(mx, float(c[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, c[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.f.name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def visible_index(local_rank):
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [x.strip() for x in vis.split(",")]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle sample
+# ---------------------------------------------------------------------------
+
+def oracle_sample(w, reps=1):
+    """Times the oracle on one chunk through one layer of the step (with its
+    predecessor K/V) and scales to a full steady-state step.  Returns
+    (frames/s extrapolated, seconds per sample, threads)."""
+    import numpy as np
+
+    import synth
+    from oracle import dit
+
+    m1 = synth.truncated(w, 1).model
+    q = w.queue
+    p = synth.make_params(m1)
+    text = synth.make_text(m1)
+    fn = dit.make_velocity_fn(p, text, m1, q.T)   # prompt K/V: once per prompt, untimed
+    lat = synth.make_noise(m1, q, 0).astype(np.float64)
+    rng = np.random.default_rng(0)
+    Lc = q.tokens_per_chunk(m1)
+    kv = [(rng.standard_normal((Lc, m1.dim)) * 0.5, rng.standard_normal((Lc, m1.dim)) * 0.5)]
+    times = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        fn([lat], [q.T // 2], [5], kv, None)
+        times.append(time.perf_counter() - t0)
+    t = min(times)
+    per_step = t * q.T * w.model.n_layers      # every queued chunk, every layer
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        threads = os.cpu_count() or 1
+    return q.frames_per_chunk / per_step, t, threads
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    vals = []
+    t_sample = 0.0
+    threads = 1
+    for i in range(args.warmup + args.steps):
+        v, t_sample, threads = oracle_sample(w)
+        if i >= args.warmup:
+            vals.append(v)
+    v = statistics.median(vals)
+    sample = (f"1 chunk x 1 layer of the {w.name} step (with its predecessor K/V), "
+              f"{t_sample:.1f} s each, scaled by T x layers = {w.queue.T * w.model.n_layers}")
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.queue.frames_per_chunk / v * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, w):
+    import numpy as np
+    import torch
+
+    from chunked_fifo_denoising_b200 import Model, Queue
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    m, q = w.model, w.queue
+    T = q.T
+    occ = T
+    stream = torch.cuda.current_stream()
+    # random-init weights on the device, N(0, 0.02^2), seeded per rank
+    g = torch.Generator(device="cuda").manual_seed(1000 + rank)
+    import synth
+    model = Model(m, "bf16", stream=stream)
+    for name, shape, per_layer in synth.param_specs(m):
+        for l in range(m.n_layers if per_layer else 1):
+            t = torch.randn(shape, generator=g, device="cuda") * 0.02
+            model.set_param(name, t, l)
+            del t
+    text = torch.randn((m.text_len, m.text_in_dim), generator=g, device="cuda")
+    n_chunks = T - 1 + args.warmup + args.steps + args.e2e_steps + 2
+    queue = Queue(model, text, T, q.frames_per_chunk, q.lat_h, q.lat_w, n_chunks,
+                  ready_capacity=2, seed=3 + rank)
+    out = torch.empty(queue.chunk_shape, device="cuda")
+    # fill: T-1 steps bring the queue to full occupancy (untimed)
+    for _ in range(T - 1):
+        queue.step(None)
+        queue.try_pop(out)
+    queue.sync()
+    info = queue.inspect()
+    assert info["n"] == occ, info
+    for _ in range(args.warmup):
+        queue.step(None)
+        queue.pop(out)
+    queue.sync()
+    # timed region: K full steps, per-kernel events on the queue's stream
+    queue.set_timing(True)
+    clocks = Clocks(visible_index(local))
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        queue.step(None)
+        queue.pop(out)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ck = clocks.stop()
+    queue.sync()
+    ms = e0.elapsed_time(e1)
+    kt = queue.timing()
+    queue.set_timing(False)
+    # end to end through the public API with host buffers (H2D noise, D2H chunk)
+    hn = torch.randn(queue.chunk_shape, generator=torch.Generator().manual_seed(rank)).pin_memory()
+    ho = torch.empty(queue.chunk_shape).pin_memory()
+    torch.cuda.synchronize()
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(args.e2e_steps):
+        queue.step(hn)
+        queue.pop(ho)
+    f1.record(stream)
+    torch.cuda.synchronize()
+    ms_e2e = f0.elapsed_time(f1)
+    queue.sync()
+    # max over ranks
+    tmax = torch.tensor([ms, ms_e2e], device="cuda", dtype=torch.float64)
+    if dist is not None:
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+    ms, ms_e2e = float(tmax[0]), float(tmax[1])
+    frames = q.frames_per_chunk
+    value = world * args.steps * frames / (ms / 1e3)
+    e2e_value = world * args.e2e_steps * frames / (ms_e2e / 1e3)
+    pk = peaks()
+    flops = step_flops(m, q, occ)
+    ms_step = ms / args.steps
+    peak_tf = pk["bf16_tflops_sustained"]
+    gemm = kt["gemm"]
+    attn = kt["self_attention"]
+    launches = sum(v["launches"] for v in kt.values())
+    roof = {"bound": "tensor", "kernel": "gemm_tc (tcgen05 GEMM, all fused epilogues)",
+            "achieved": gemm["flops"] / (gemm["ms"] / 1e3) / 1e12 if gemm["ms"] > 0 else None,
+            "peak": peak_tf, "unit": "TFLOP/s",
+            "peak_source": f"{pk['_source']} bf16_tflops_sustained (kernel timed inside a long step)",
+            "traffic": None}
+    if roof["achieved"]:
+        roof["frac"] = roof["achieved"] / peak_tf
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: seeded N(0,1) noise and prompt, N(0,0.02^2) random-init weights",
+            "config": {"workload": w.name, "T": T, "occupancy": occ, "chunk_tokens": q.tokens_per_chunk(m),
+                       "tokens_per_step": occ * q.tokens_per_chunk(m), "frames_per_step": frames,
+                       "layers": m.n_layers, "dim": m.dim, "ffn": m.ffn_dim, "heads": m.n_heads,
+                       "text_tokens": m.text_len, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (fp32 residual stream alone is "
+                             f"{occ * q.tokens_per_chunk(m) * m.dim * 4 / 1e6:.0f} MB)"},
+            "pct_bf16_peak": 100.0 * flops / (ms_step / 1e3) / (peak_tf * 1e12),
+            "step_tflop": flops / 1e12,
+            "roofline": roof,
+            "kernels": {k: {"ms_per_step": v["ms"] / args.steps, "launches_per_step": v["launches"] / args.steps,
+                            "tflops": (v["flops"] / (v["ms"] / 1e3) / 1e12) if v["ms"] > 0 and v["flops"] else None,
+                            "gbs": (v["bytes"] / (v["ms"] / 1e3) / 1e9) if v["ms"] > 0 and v["bytes"] else None}
+                        for k, v in kt.items() if v["launches"]},
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(hn.numel() * 4),
+                    "d2h_bytes_per_step": int(ho.numel() * 4), "steps": args.e2e_steps},
+            "gpu_launches": launches, "clocks": ck}
+    if attn["ms"] > 0:
+        line["self_attention_tflops"] = attn["flops"] / (attn["ms"] / 1e3) / 1e12
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, t, threads = oracle_sample(w)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
+                                "sample": f"1 chunk x 1 layer of the step ({t:.1f} s), scaled by "
+                                          f"T x layers = {T * m.n_layers}; float64 numpy"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    model.close()
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="wan1.3b_480p")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    import synth
+    w = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

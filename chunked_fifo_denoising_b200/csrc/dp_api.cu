@@ -778,7 +778,8 @@ dp_status dp_queue_step(dp_queue* q, const float* noise, dp_loc loc) {
   if (pl.head_pred == kPredCache && q->cache_id != pl.head - 1)
     return fail(DP_ERR_STATE, "persisted K/V belong to chunk %lld, head needs chunk %lld",
                 q->cache_id, pl.head - 1);
-  if (q->timer.on) DP_TRY(q->timer.collect());
+  // timing records are read back lazily (on query, or when many are pending)
+  if (q->timer.on && q->timer.pending.size() > 16384) DP_TRY(q->timer.collect());
   dp_model* m = q->m;
   cudaStream_t s = m->stream;
   if (pl.push) {

@@ -109,6 +109,20 @@ dp_status dp_op_attention(const dp_attn_args* a, void* stream) {
   return DP_OK;
 }
 
+dp_status dp_op_check(void* stream) {
+  clear_error();
+  DP_CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  int* w = op_status_word();
+  if (!w) return fail(DP_ERR_CUDA, "status word unavailable");
+  int v = 0;
+  DP_CK(cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost));
+  if (v) {
+    DP_CK(cudaMemset(w, 0, sizeof(int)));
+    return fail(DP_ERR_KERNEL, "a kernel gave up a bounded wait (status 0x%x)", v);
+  }
+  return DP_OK;
+}
+
 dp_status dp_op_layernorm_mod(const dp_ln_args* a, void* stream) {
   clear_error();
   if (!a || !a->x || !a->out) return fail(DP_ERR_INVALID_ARG, "NULL argument");

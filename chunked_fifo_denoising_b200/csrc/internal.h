@@ -91,6 +91,9 @@ cudaError_t add_layer_tables(const float* m, const float* table, int T, int L, i
 cudaError_t normal_fill(unsigned long long seed, unsigned long long a, unsigned long long b,
                         float* out, long long n, cudaStream_t s);
 
+// Device status word of kernels launched from the single-kernel entry points.
+int* op_status_word();
+
 cudaError_t convert_f32_to_bf16(const float* in, bf16* out, long long n, cudaStream_t s);
 cudaError_t convert_bf16_to_f32(const bf16* in, float* out, long long n, cudaStream_t s);
 // strided 2-D copy/convert of a [rows][cols] block between float/bf16 buffers

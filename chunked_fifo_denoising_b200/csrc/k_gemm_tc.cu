@@ -13,6 +13,7 @@
 //               next tile's MMAs overlap this tile's epilogue.
 // Tiles are walked row-block-major so the CTAs in flight share A row blocks
 // through L2 while W stays L2-resident.  Every mbarrier wait is bounded.
+#include <cstring>
 #include <mutex>
 
 #include "tc_common.cuh"
@@ -39,74 +40,36 @@ __device__ __forceinline__ void store_bf16x32(bf16* dst, const float (&v)[32]) {
   }
 }
 
-// Fused epilogue for 32 consecutive columns [col0, col0+32) of one row.
-__device__ __forceinline__ void epilogue32(const EpiParams& e, int row, int col0, float (&v)[32]) {
-  if (e.bias) {
-    const float4* b4 = reinterpret_cast<const float4*>(e.bias + col0);
+// Bias (and activation) for `n` consecutive columns starting at col0; columns
+// at or beyond N read no bias.
+template <int NV>
+__device__ __forceinline__ void add_bias(const EpiParams& e, int col0, int N, float (&v)[NV]) {
+  if (!e.bias) return;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float4 b = b4[i];
+  for (int i = 0; i < NV / 4; ++i) {
+    if (col0 + 4 * i < N) {
+      const float4 b = reinterpret_cast<const float4*>(e.bias + col0)[i];
       v[4 * i] += b.x;
       v[4 * i + 1] += b.y;
       v[4 * i + 2] += b.z;
       v[4 * i + 3] += b.w;
     }
   }
-  switch (e.mode) {
-    case EPI_GELU:
+}
+
+// One 128-byte row (8 chunks of 16 bytes) of a 128-byte-swizzled staging box:
+// chunk j of row r lives at chunk position j ^ (r % 8), so the 8 rows a
+// quarter-warp writes at once fall in distinct banks.
+__device__ __forceinline__ void stage_row(uint8_t* box, int r, const uint32_t (&w)[32]) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) v[i] = gelu_erf(v[i]);
-      store_bf16x32((bf16*)e.out + (long long)row * e.ldo + col0, v);
-      break;
-    case EPI_STORE:
-      if (e.out_f32) {
-        float4* o = reinterpret_cast<float4*>((float*)e.out + (long long)row * e.ldo + col0);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) o[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-      } else {
-        store_bf16x32((bf16*)e.out + (long long)row * e.ldo + col0, v);
-        if (e.cache && row >= e.cache_row0 && row < e.cache_row0 + e.cache_rows &&
-            col0 >= e.cache_col0)
-          store_bf16x32((bf16*)e.cache + (long long)(row - e.cache_row0) * e.ldc + (col0 - e.cache_col0), v);
-      }
-      break;
-    case EPI_RESID:
-    case EPI_RESID_GATED: {
-      float4* x = reinterpret_cast<float4*>(e.resid + (long long)row * e.ldr + col0);
-      const float4* g = nullptr;
-      if (e.mode == EPI_RESID_GATED) {
-        const int c = row / e.rows_per_chunk;
-        const long long sel = e.chunk_sel ? e.chunk_sel[c] : c;
-        g = reinterpret_cast<const float4*>(e.gate + sel * e.gate_stride + col0);
-      }
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float4 r = x[i];
-        if (g) {
-          const float4 gg = g[i];
-          r.x = fmaf(gg.x, v[4 * i], r.x);
-          r.y = fmaf(gg.y, v[4 * i + 1], r.y);
-          r.z = fmaf(gg.z, v[4 * i + 2], r.z);
-          r.w = fmaf(gg.w, v[4 * i + 3], r.w);
-        } else {
-          r.x += v[4 * i];
-          r.y += v[4 * i + 1];
-          r.z += v[4 * i + 2];
-          r.w += v[4 * i + 3];
-        }
-        x[i] = r;
-      }
-      break;
-    }
-    case EPI_EULER: {
-      const float ds = e.dsig[row / e.rows_per_chunk];
-#pragma unroll 4
-      for (int i = 0; i < 32; ++i) e.ring[euler_index(e, row, col0 + i, e.rows_per_chunk)] += ds * v[i];
-      break;
-    }
-    default:
-      break;
-  }
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<uint4*>(box + r * 128 + ((j ^ (r & 7)) << 4)) =
+        make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&p);
 }
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
@@ -116,13 +79,19 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+struct GemmMaps {
+  CUtensorMap a, b;    // operands
+  CUtensorMap out;     // STORE/GELU output (bf16 box 64x32 or fp32 box 32x32)
+  CUtensorMap res;     // fp32 residual stream for the reduce-add epilogues
+};
+
 template <int BN, int STAGES>
 __global__ void __launch_bounds__(192, 1)
-gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-               int M, int N, int K, EpiParams e, int* status) {
+gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiParams e, int* status) {
   constexpr uint32_t A_BYTES = BM * BK * 2;
   constexpr uint32_t B_BYTES = BN * BK * 2;
   constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr uint32_t STG_OFF = STAGES * STAGE_BYTES;  // 4 warps x 2 staging boxes of 4 KB
   constexpr uint32_t TMEM_COLS = 2 * BN;
   constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, 0, 0);
 
@@ -156,8 +125,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
     tmem_relinquish();
   }
   if (warp == 0 && lane == 0) {
-    prefetch_tmap(&tmA);
-    prefetch_tmap(&tmB);
+    prefetch_tmap(&maps.a);
+    prefetch_tmap(&maps.b);
   }
   tc_fence_before();
   __syncthreads();
@@ -180,8 +149,8 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
           }
           uint8_t* sa = smem + stage * STAGE_BYTES;
           mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
-          tma_load_2d(sa, &tmA, kb * BK, m0, &full_bar[stage]);
-          tma_load_2d(sa + A_BYTES, &tmB, kb * BK, n0, &full_bar[stage]);
+          tma_load_2d(sa, &maps.a, kb * BK, m0, &full_bar[stage]);
+          tma_load_2d(sa + A_BYTES, &maps.b, kb * BK, n0, &full_bar[stage]);
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -235,25 +204,117 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ 
   } else {
     // ---------------- epilogue (warps 2..5) ----------------
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
-    const int rloc = quad * 32 + lane;
+    uint8_t* stg = smem + STG_OFF + (warp - 2) * 8192;
+    uint32_t sb = 0;            // staging boxes used by this warp so far
+    const bool bf16_out = (e.mode == EPI_STORE && !e.out_f32) || e.mode == EPI_GELU;
+    const bool reduce = e.mode == EPI_RESID || e.mode == EPI_RESID_GATED;
     int it = 0;
     for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
       const int buf = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
-      if (!mbar_wait(&tfull_bar[buf], acc_phase, &abort_flag, status, ST_TIMEOUT_GEMM)) break;
+      // warp-uniform: the TMEM loads below are warp-collective
+      const bool waited = mbar_wait(&tfull_bar[buf], acc_phase, &abort_flag, status, ST_TIMEOUT_GEMM);
+      if (!__all_sync(0xffffffffu, waited)) break;
       tc_fence_after();
       const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
-      const int row = m0 + rloc;
+      const int row_base = m0 + quad * 32;
+      const int row = row_base + lane;
+      const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN;
+      if (bf16_out) {
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        float v[32];
-        tmem_ld32(tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + c * 32, v);
-        const int col0 = n0 + c * 32;
-        if (row < M && col0 < N) epilogue32(e, row, col0, v);
+        for (int g = 0; g < BN / 64; ++g) {
+          const int col0 = n0 + g * 64;
+          if (col0 >= N) break;  // uniform
+          float v[64];
+          float* v0 = v;
+          tmem_ld32(tbase + g * 64, *reinterpret_cast<float(*)[32]>(v0));
+          tmem_ld32(tbase + g * 64 + 32, *reinterpret_cast<float(*)[32]>(v0 + 32));
+          add_bias<64>(e, col0, N, v);
+          if (e.mode == EPI_GELU) {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) v[i] = gelu_erf(v[i]);
+          }
+          uint32_t w[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = pack_bf16(v[2 * i], v[2 * i + 1]);
+          if (e.cache && row < M && row >= e.cache_row0 && row < e.cache_row0 + e.cache_rows &&
+              col0 >= e.cache_col0) {
+            uint4* d = reinterpret_cast<uint4*>((bf16*)e.cache + (long long)(row - e.cache_row0) * e.ldc +
+                                                (col0 - e.cache_col0));
+            const int nchunk = min(8, (N - col0) / 8);
+            for (int j = 0; j < nchunk; ++j) d[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+          }
+          uint8_t* box = stg + (sb & 1) * 4096;
+          if (lane == 0) bulk_wait_read<1>();  // the box written two rounds ago has been read
+          __syncwarp();
+          stage_row(box, lane, w);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&maps.out, col0, row_base, box);
+            bulk_commit();
+          }
+          ++sb;
+        }
+      } else if (e.mode == EPI_EULER) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          float v[32];
+          tmem_ld32(tbase + c * 32, v);
+          const int col0 = n0 + c * 32;
+          if (row < M && col0 < N) {
+            add_bias<32>(e, col0, N, v);
+            const float ds = e.dsig[row / e.rows_per_chunk];
+            for (int i = 0; i < 32; ++i) e.ring[euler_index(e, row, col0 + i, e.rows_per_chunk)] += ds * v[i];
+          }
+        }
+      } else {
+        // fp32 results: plain store (residual stream init) or reduce-add into it
+        const int grow = row < M ? row : M - 1;  // rows past M are clipped by TMA; keep lookups in range
+        const float* gate = nullptr;
+        if (e.mode == EPI_RESID_GATED) {
+          const int c = grow / e.rows_per_chunk;
+          const long long sel = e.chunk_sel ? e.chunk_sel[c] : c;
+          gate = e.gate + sel * e.gate_stride;
+        }
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          const int col0 = n0 + c * 32;
+          if (col0 >= N) break;  // uniform
+          float v[32];
+          tmem_ld32(tbase + c * 32, v);
+          add_bias<32>(e, col0, N, v);
+          if (gate) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float4 gg = reinterpret_cast<const float4*>(gate + col0)[i];
+              v[4 * i] *= gg.x;
+              v[4 * i + 1] *= gg.y;
+              v[4 * i + 2] *= gg.z;
+              v[4 * i + 3] *= gg.w;
+            }
+          }
+          uint32_t w[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i]);
+          uint8_t* box = stg + (sb & 1) * 4096;
+          if (lane == 0) bulk_wait_read<1>();
+          __syncwarp();
+          stage_row(box, lane, w);
+          fence_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            if (reduce) tma_reduce_add_2d(&maps.res, col0, row_base, box);
+            else tma_store_2d(&maps.out, col0, row_base, box);
+            bulk_commit();
+          }
+          ++sb;
+        }
       }
       tc_fence_before();
       mbar_arrive(&tempty_bar[buf]);
     }
+    if (lane == 0) bulk_wait_all();  // stores and reductions have landed
   }
   tc_fence_before();
   __syncthreads();
@@ -297,19 +358,28 @@ int sm_count() {
 
 }  // namespace
 
+// Row-major [rows][cols] (row stride `ld` elements) of bf16 or fp32, boxes of
+// box_rows x box_cols with the 128-byte swizzle (box_cols * element = 128 B).
+static bool make_tmap(CUtensorMap* map, bool f32, const void* base, long long rows, long long cols,
+                      long long ld, int box_rows, int box_cols) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const int es = f32 ? 4 : 2;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld * es};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                  const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 // bf16 [rows][cols] row-major with row stride `ld` elements; box box_rows x 64.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, long long rows, long long cols, long long ld,
                     int box_rows, int box_cols) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  cuuint64_t strides[1] = {(cuuint64_t)ld * 2};
-  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS;
+  return make_tmap(map, false, base, rows, cols, ld, box_rows, box_cols);
 }
 
 bool gemm_tc_supported(long long lda, int M, int N, int K) {
@@ -319,7 +389,7 @@ bool gemm_tc_supported(long long lda, int M, int N, int K) {
 template <int BN, int STAGES>
 static cudaError_t launch_tc(const bf16* A, long long lda, const bf16* W, int M, int N, int K,
                              const EpiParams& e, int* status, cudaStream_t s) {
-  constexpr int SMEM = STAGES * (BM * BK * 2 + BN * BK * 2) + 1024;
+  constexpr int SMEM = STAGES * (BM * BK * 2 + BN * BK * 2) + 4 * 8192 + 1024;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
@@ -327,12 +397,23 @@ static cudaError_t launch_tc(const bf16* A, long long lda, const bf16* W, int M,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   });
   if (attr_err != cudaSuccess) return attr_err;
-  CUtensorMap ta, tb;
-  if (!make_tmap_bf16(&ta, A, M, K, lda, BM, BK)) return cudaErrorInvalidValue;
-  if (!make_tmap_bf16(&tb, W, N, K, K, BN, BK)) return cudaErrorInvalidValue;
+  GemmMaps maps;
+  memset(&maps, 0, sizeof(maps));
+  if (!make_tmap(&maps.a, false, A, M, K, lda, BM, BK)) return cudaErrorInvalidValue;
+  if (!make_tmap(&maps.b, false, W, N, K, K, BN, BK)) return cudaErrorInvalidValue;
+  if (e.mode == EPI_GELU || (e.mode == EPI_STORE && !e.out_f32)) {
+    if (!make_tmap(&maps.out, false, e.out, M, N, e.ldo, 32, 64)) return cudaErrorInvalidValue;
+  } else if (e.mode == EPI_STORE) {
+    if (!make_tmap(&maps.out, true, e.out, M, N, e.ldo, 32, 32)) return cudaErrorInvalidValue;
+  } else if (e.mode == EPI_RESID || e.mode == EPI_RESID_GATED) {
+    if (!make_tmap(&maps.res, true, e.resid, M, N, e.ldr, 32, 32)) return cudaErrorInvalidValue;
+  } else if (e.mode != EPI_EULER) {
+    return cudaErrorInvalidValue;
+  }
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = tiles < sm_count() ? tiles : sm_count();
-  gemm_tc_kernel<BN, STAGES><<<grid, 192, SMEM, s>>>(ta, tb, M, N, K, e, status);
+  if (!status) status = op_status_word();
+  gemm_tc_kernel<BN, STAGES><<<grid, 192, SMEM, s>>>(maps, M, N, K, e, status);
   return cudaGetLastError();
 }
 

@@ -5,6 +5,23 @@
 
 namespace dp {
 
+static __device__ int g_op_status;
+
+int* op_status_word() {
+  // the symbol's device address differs per device: look it up per device
+  static int* ptr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (!ptr[dev] && cudaGetSymbolAddress(reinterpret_cast<void**>(&ptr[dev]), g_op_status) != cudaSuccess) {
+    cudaGetLastError();
+    ptr[dev] = nullptr;
+  }
+  return ptr[dev];
+}
+
 // ---------------------------------------------------------------------------
 // LayerNorm (no affine, biased variance, eps 1e-6) + adaLN shift/scale.
 // One 128-thread block per row, 128-bit loads of x; the row stays in

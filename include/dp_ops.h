@@ -100,6 +100,11 @@ typedef struct {
 } dp_ln_args;
 DP_API dp_status dp_op_layernorm_mod(const dp_ln_args* a, void* stream);
 
+/* Waits for `stream`, then reads and clears the status word that the
+ * tensor-core kernels of the calls above set when one of their bounded waits
+ * gives up (they then skip the rest of their work).  DP_ERR_KERNEL if set. */
+DP_API dp_status dp_op_check(void* stream);
+
 #ifdef __cplusplus
 }
 #endif

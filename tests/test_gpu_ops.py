@@ -65,7 +65,7 @@ def run_gemm(A, W, bias, epi, out=None, resid=None, gate=None, sel=None, rpc=1, 
             cache.data_ptr(), cache_row0, cache_rows, cache_col0, cache.stride(0))
     st = B.dp_op_gemm(a, torch.cuda.current_stream().cuda_stream)
     assert st == 0, B.dp_last_error()
-    torch.cuda.synchronize()
+    assert B.dp_op_check(torch.cuda.current_stream().cuda_stream) == 0, B.dp_last_error()
 
 
 @pytest.mark.parametrize("M,N,K", [(300, 256, 128), (129, 64, 64), (1000, 384, 192),
@@ -174,7 +174,7 @@ def run_attn(q, k, v, n_chunks, Lq, H, hd, Lk, kv_chunk_rows, pred_in_batch, kp=
     a.out, a.ldo = out.data_ptr(), out.stride(0)
     st = B.dp_op_attention(a, torch.cuda.current_stream().cuda_stream)
     assert st == 0, B.dp_last_error()
-    torch.cuda.synchronize()
+    assert B.dp_op_check(torch.cuda.current_stream().cuda_stream) == 0, B.dp_last_error()
     return out
 
 
