@@ -8,15 +8,18 @@
 // buffer through one online softmax; the buffers are never concatenated.  The
 // same kernel with one shared buffer is the cross-attention to the prompt.
 //
-// CTA = one 128-query tile of one (chunk, head); 6 warps:
-//   warp 0      TMA producer: Q once, then K and V tiles (128 keys) into a
-//               2-stage ring, each tile from whichever buffer it belongs to
-//   warp 1      TMEM owner + MMA issuer: S_j = Q K_j^T (M=128, N=128, K=hd)
-//               into one of two TMEM S buffers, O += P_j V_j (N=hd, K=128)
-//   warps 2..5  softmax, thread = query row: S row from TMEM, mask, online
-//               max/sum in the log2 domain, P (bf16) into swizzled smem;
-//               O is rescaled in TMEM only when a row maximum grows by more
-//               than 2^8 (exact: the final division uses the same reference)
+// CTA = 256 queries (two 128-row tiles A and B) of one (chunk, head), 10 warps:
+//   warp 0      TMA producer: Q_A, Q_B once; K and V tiles of 128 keys into two
+//               2-stage rings, each tile from whichever buffer it belongs to
+//   warp 1      TMEM owner + MMA issuer, tiles ping-ponged on the tensor core:
+//               S_X = Q_X K_j^T (M=128, N=128, K=hd) into TMEM, then
+//               O_X += P_X V_j with P_X read from TMEM (the TS form)
+//   warps 2..5  softmax of tile A, warps 6..9 softmax of tile B; thread = query
+//               row: S row from TMEM, online max/sum in the log2 domain, P as
+//               bf16 written back over S in TMEM; O is rescaled in TMEM only when
+//               a row maximum grows by more than 2^8 (exact: the final division
+//               uses the same reference)
+// TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+hd) O_B [256+hd,256+2hd).
 // Every mbarrier wait is bounded.
 #include <mutex>
 
@@ -37,17 +40,15 @@ template <int HD>
 struct Cfg {
   static constexpr int NSUB = HD / 64;              // 64-column (128-byte) sub-tiles
   static constexpr uint32_t SUB_BYTES = 128 * 128;  // 128 rows x 128 bytes
-  static constexpr uint32_t Q_BYTES = NSUB * SUB_BYTES;
-  static constexpr uint32_t K_BYTES = NSUB * SUB_BYTES;
-  static constexpr uint32_t V_BYTES = NSUB * SUB_BYTES;
-  static constexpr uint32_t P_BYTES = 2 * SUB_BYTES;  // 128 queries x 128 keys bf16
-  static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_K = Q_BYTES;                 // 2 stages
-  static constexpr uint32_t OFF_V = OFF_K + 2 * K_BYTES;     // 2 stages
-  static constexpr uint32_t OFF_P = OFF_V + 2 * V_BYTES;     // 2 buffers
-  static constexpr uint32_t SMEM = OFF_P + 2 * P_BYTES + 1024;
-  static constexpr uint32_t TMEM_COLS = 512;                 // S0, S1 (128 each), O (hd)
-  static constexpr uint32_t O_COL = 256;
+  static constexpr uint32_t T_BYTES = NSUB * SUB_BYTES;  // one 128-row tile of Q, K or V
+  static constexpr uint32_t OFF_QA = 0;
+  static constexpr uint32_t OFF_QB = T_BYTES;
+  static constexpr uint32_t OFF_K = 2 * T_BYTES;             // 2 stages
+  static constexpr uint32_t OFF_V = OFF_K + 2 * T_BYTES;     // 2 stages
+  static constexpr uint32_t SMEM = OFF_V + 2 * T_BYTES + 1024;
+  static constexpr uint32_t TMEM_COLS = 512;
+  __device__ static constexpr uint32_t s_col(int X) { return X ? 128u : 0u; }
+  __device__ static constexpr uint32_t o_col(int X) { return 256u + (X ? (uint32_t)HD : 0u); }
 };
 
 struct AttnMaps {
@@ -65,6 +66,11 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, w);
 }
 
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const unsigned long long t0 = globaltimer();
   while (!mbar_try_wait(bar, parity)) {
@@ -73,18 +79,21 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
 }
 
 template <int HD>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status) {
   using C = Cfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t q_full, k_full[2], v_full[2], kv_empty[2], s_full[2], s_empty[2], p_full[2],
+  __shared__ uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2],
       pv_done[2], done_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, h = blockIdx.y, c = blockIdx.z;
+  const int h = blockIdx.y, c = blockIdx.z;
+  const int q0 = blockIdx.x * 2 * BQ;        // first query of tile A within the chunk
+  const bool has_b = q0 + BQ < p.Lq;         // tile B holds at least one query
+  const int qrow0 = c * p.Lq + q0;
   // key sources of this chunk
   int n_p = 0;
   bool pred_cache = false;
@@ -97,16 +106,15 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
   const int n_o = p.Lk;
   const int tiles_p = (n_p + BKV - 1) / BKV;
   const int nt = tiles_p + (n_o + BKV - 1) / BKV;
-  const int qrow0 = c * p.Lq + qt * BQ;
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&k_full[i], 1);
+      mbar_init(&k_empty[i], 1);
       mbar_init(&v_full[i], 1);
-      mbar_init(&kv_empty[i], 1);
+      mbar_init(&v_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&s_empty[i], 128);
       mbar_init(&p_full[i], 128);
       mbar_init(&pv_done[i], 1);
     }
@@ -127,15 +135,16 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       const int col0 = h * HD;
-      mbar_arrive_expect_tx(&q_full, C::Q_BYTES);
+      mbar_arrive_expect_tx(&q_full, (has_b ? 2 : 1) * C::T_BYTES);
 #pragma unroll
-      for (int s = 0; s < C::NSUB; ++s)
-        tma_load_2d(smem + C::OFF_Q + s * C::SUB_BYTES, &maps.q, col0 + 64 * s, qrow0, &q_full);
-      uint32_t issued = 0, issued_par = 0;
+      for (int s = 0; s < C::NSUB; ++s) {
+        tma_load_2d(smem + C::OFF_QA + s * C::SUB_BYTES, &maps.q, col0 + 64 * s, qrow0, &q_full);
+        if (has_b) tma_load_2d(smem + C::OFF_QB + s * C::SUB_BYTES, &maps.q, col0 + 64 * s, qrow0 + BQ, &q_full);
+      }
+      uint32_t issued_k = 0, issued_v = 0, par = 0;
       for (int j = 0; j < nt; ++j) {
         const int st = j & 1;
         const uint32_t use = (uint32_t)(j >> 1);
-        if (use > 0 && !mbar_wait(&kv_empty[st], (use - 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
         const CUtensorMap* mk;
         const CUtensorMap* mv;
         int row;
@@ -154,24 +163,26 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
           mv = &maps.v;
           row = (int)(c * p.kv_chunk_rows) + (j - tiles_p) * BKV;
         }
-        mbar_arrive_expect_tx(&k_full[st], C::K_BYTES);
+        if (use > 0 && !mbar_wait(&k_empty[st], (use - 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
+        mbar_arrive_expect_tx(&k_full[st], C::T_BYTES);
 #pragma unroll
         for (int s = 0; s < C::NSUB; ++s)
-          tma_load_2d(smem + C::OFF_K + st * C::K_BYTES + s * C::SUB_BYTES, mk, col0 + 64 * s, row, &k_full[st]);
-        mbar_arrive_expect_tx(&v_full[st], C::V_BYTES);
+          tma_load_2d(smem + C::OFF_K + st * C::T_BYTES + s * C::SUB_BYTES, mk, col0 + 64 * s, row, &k_full[st]);
+        issued_k |= 1u << st;
+        par = (par & ~(1u << st)) | ((use & 1u) << st);
+        if (use > 0 && !mbar_wait(&v_empty[st], (use - 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
+        mbar_arrive_expect_tx(&v_full[st], C::T_BYTES);
 #pragma unroll
         for (int s = 0; s < C::NSUB; ++s)
-          tma_load_2d(smem + C::OFF_V + st * C::V_BYTES + s * C::SUB_BYTES, mv, col0 + 64 * s, row, &v_full[st]);
-        issued |= 1u << st;
-        issued_par = (issued_par & ~(1u << st)) | ((use & 1u) << st);
+          tma_load_2d(smem + C::OFF_V + st * C::T_BYTES + s * C::SUB_BYTES, mv, col0 + 64 * s, row, &v_full[st]);
+        issued_v |= 1u << st;
       }
-      if (abort_flag) {
+      if (abort_flag) {  // let copies in flight land before the CTA exits
         drain_wait(&q_full, 0);
-        for (int st = 0; st < 2; ++st)
-          if (issued & (1u << st)) {
-            drain_wait(&k_full[st], (issued_par >> st) & 1u);
-            drain_wait(&v_full[st], (issued_par >> st) & 1u);
-          }
+        for (int st = 0; st < 2; ++st) {
+          if (issued_k & (1u << st)) drain_wait(&k_full[st], (par >> st) & 1u);
+          if (issued_v & (1u << st)) drain_wait(&v_full[st], (par >> st) & 1u);
+        }
       }
     }
   } else if (warp == 1) {
@@ -179,147 +190,142 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
       // ---------------- MMA issuer ----------------
       constexpr uint32_t IDESC_S = idesc_bf16_f32(BQ, BKV, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(BQ, HD, 0, 1);
-      const uint32_t sQ = smem_u32(smem + C::OFF_Q);
-      bool ok = mbar_wait(&q_full, 0, &abort_flag, status, ST_TIMEOUT_ATTN);
-      auto issue_s = [&](int j) -> bool {
-        const int st = j & 1;
-        if (!mbar_wait(&k_full[st], (j >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) return false;
-        if (j >= 2 && !mbar_wait(&s_empty[st], ((j >> 1) - 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN))
-          return false;
-        tc_fence_after();
-        const uint32_t sK = smem_u32(smem + C::OFF_K + st * C::K_BYTES);
+      auto issue_s = [&](int X, int j) {
+        const uint32_t sQ = smem_u32(smem + (X ? C::OFF_QB : C::OFF_QA));
+        const uint32_t sK = smem_u32(smem + C::OFF_K + (j & 1) * C::T_BYTES);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::SUB_BYTES + (kk & 3) * 32;
-          mma_bf16_ss(tmem + st * 128, desc_sw128(sQ + off, 16, 1024), desc_sw128(sK + off, 16, 1024),
+          mma_bf16_ss(tmem + C::s_col(X), desc_sw128(sQ + off, 16, 1024), desc_sw128(sK + off, 16, 1024),
                       IDESC_S, kk > 0);
         }
-        mma_commit(&s_full[st]);
-        return true;
+        mma_commit(&s_full[X]);
       };
-      if (ok) ok = issue_s(0);
-      for (int j = 0; j < nt && ok; ++j) {
-        if (j + 1 < nt && !issue_s(j + 1)) break;
-        const int b = j & 1;
-        if (!mbar_wait(&p_full[b], (j >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
-        if (!mbar_wait(&v_full[b], (j >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
-        tc_fence_after();
-        const uint32_t sP = smem_u32(smem + C::OFF_P + b * C::P_BYTES);
-        const uint32_t sV = smem_u32(smem + C::OFF_V + b * C::V_BYTES);
+      auto issue_pv = [&](int X, int j) {
+        const uint32_t sV = smem_u32(smem + C::OFF_V + (j & 1) * C::T_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk) {
-          const uint64_t ad = desc_sw128(sP + (kk >> 2) * C::SUB_BYTES + (kk & 3) * 32, 16, 1024);
-          // V is MN-major: 16 keys = 2 atoms of 8 rows (2048 B); hd groups of 64 are SUB_BYTES apart
-          const uint64_t bd = desc_sw128(sV + kk * 2048, C::SUB_BYTES, 1024);
-          mma_bf16_ss(tmem + C::O_COL, ad, bd, IDESC_O, (j | kk) != 0);
+        for (int kk = 0; kk < BKV / 16; ++kk)  // 16 keys = 8 TMEM columns of packed P; 2 atoms of V
+          mma_bf16_ts(tmem + C::o_col(X), tmem + C::s_col(X) + kk * 8,
+                      desc_sw128(sV + kk * 2048, C::SUB_BYTES, 1024), IDESC_O, (j | kk) != 0);
+        mma_commit(&pv_done[X]);
+      };
+      bool ok = mbar_wait(&q_full, 0, &abort_flag, status, ST_TIMEOUT_ATTN) &&
+                mbar_wait(&k_full[0], 0, &abort_flag, status, ST_TIMEOUT_ATTN);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        if (has_b) issue_s(1, 0);
+        mma_commit(&k_empty[0]);
+      }
+      for (int j = 0; j < nt && ok; ++j) {
+        const bool next = j + 1 < nt;
+        if (!mbar_wait(&v_full[j & 1], (j >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
+        if (!mbar_wait(&p_full[0], j & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
+        tc_fence_after();
+        issue_pv(0, j);
+        if (next) {
+          if (!mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
+          tc_fence_after();
+          issue_s(0, j + 1);
         }
-        mma_commit(&pv_done[b]);
-        mma_commit(&kv_empty[b]);
+        if (has_b) {
+          if (!mbar_wait(&p_full[1], j & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
+          tc_fence_after();
+          issue_pv(1, j);
+        }
+        mma_commit(&v_empty[j & 1]);
+        if (next) {
+          if (has_b) issue_s(1, j + 1);
+          mma_commit(&k_empty[(j + 1) & 1]);
+        }
       }
       mma_commit(&done_bar);
       drain_wait(&done_bar, 0);
     }
     __syncwarp();
   } else {
-    // ---------------- softmax + output (warps 2..5) ----------------
-    const int quad = warp & 3;
-    const int r = quad * 32 + lane;  // query row in the tile == TMEM lane
-    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-    const float sl2 = 1.4426950408889634f / sqrtf((float)HD);  // log2(e) / sqrt(hd)
-    float m = -INFINITY, l = 0.0f;
-    bool ok = true;
-    for (int j = 0; j < nt; ++j) {
-      const int b = j & 1;
-      if (!warp_wait(&s_full[b], (j >> 1) & 1, &abort_flag, status)) { ok = false; break; }
-      tc_fence_after();
-      float s[128];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        float t[32];
-        tmem_ld32(tmem + lane_off + b * 128 + i * 32, t);
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[i * 32 + e] = t[e];
-      }
-      tc_fence_before();
-      mbar_arrive(&s_empty[b]);
-      const int valid = tile_valid(j, tiles_p, n_p, n_o);
-      float mx = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        s[i] = i < valid ? s[i] * sl2 : -INFINITY;
-        mx = fmaxf(mx, s[i]);
-      }
-      const float m_new = fmaxf(m, mx);
-      const bool want = (m == -INFINITY) || (m_new > m + 8.0f);
-      const bool resc = __any_sync(0xffffffffu, want);  // TMEM access is warp-collective
-      const float m_use = resc ? m_new : m;
-      float sum = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 128; ++i) {
-        s[i] = exp2f(s[i] - m_use);
-        sum += s[i];
-      }
-      if (j >= 2 && !warp_wait(&pv_done[b], ((j - 2) >> 1) & 1, &abort_flag, status)) {
-        ok = false;
-        break;
-      }
-      if (resc && j > 0) {
-        if (!warp_wait(&pv_done[(j - 1) & 1], ((j - 1) >> 1) & 1, &abort_flag, status)) {
-          ok = false;
-          break;
-        }
+    // ---------------- softmax + output (warps 2..9) ----------------
+    const int X = warp >= 6 ? 1 : 0;
+    if (X == 0 || has_b) {
+      const int quad = warp & 3;
+      const int r = quad * 32 + lane;  // query row in the tile == TMEM lane
+      const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+      const uint32_t tS = tmem + lane_off + C::s_col(X);
+      const uint32_t tO = tmem + lane_off + C::o_col(X);
+      const float sl2 = 1.4426950408889634f / sqrtf((float)HD);  // log2(e) / sqrt(hd)
+      float m = -INFINITY, l = 0.0f;
+      bool ok = true;
+      for (int j = 0; j < nt; ++j) {
+        if (!warp_wait(&s_full[X], j & 1, &abort_flag, status)) { ok = false; break; }
         tc_fence_after();
-        const float corr = exp2f(m - m_use);
-        l *= corr;
+        float s[128];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tmem_ld32(tS + i * 32, *reinterpret_cast<float(*)[32]>(s + i * 32));
+        const int valid = tile_valid(j, tiles_p, n_p, n_o);
+        if (valid < BKV) {
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (i >= valid) s[i] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+        const float m_new = fmaxf(m, mx * sl2);
+        const bool want = (m == -INFINITY) || (m_new > m + 8.0f);
+        const bool resc = __any_sync(0xffffffffu, want);  // TMEM access is warp-collective
+        const float m_use = resc ? m_new : m;
+        const float nm = -m_use;
+        float sum0 = 0.0f, sum1 = 0.0f;
+        uint32_t w[64];
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float a = ex2_approx(fmaf(s[2 * i], sl2, nm));
+          const float b = ex2_approx(fmaf(s[2 * i + 1], sl2, nm));
+          sum0 += a;
+          sum1 += b;
+          w[i] = pack_bf16(a, b);
+        }
+        if (resc && j > 0) {
+          // O must hold PV of every earlier tile before it is rescaled
+          if (!warp_wait(&pv_done[X], (j - 1) & 1, &abort_flag, status)) { ok = false; break; }
+          tc_fence_after();
+          const float corr = ex2_approx(m - m_use);
+          l *= corr;
+#pragma unroll 1
+          for (int i = 0; i < HD / 32; ++i) {
+            float t[32];
+            tmem_ld32(tO + i * 32, t);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) t[e] *= corr;
+            tmem_st32(tO + i * 32, t);
+          }
+        }
+        l += sum0 + sum1;
+        m = m_use;
+        // P (bf16, two keys per column) over the first 64 columns of S
+#pragma unroll
+        for (int i = 0; i < 4; ++i) tmem_st16_nowait(tS + i * 16, w + i * 16);
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[X]);
+      }
+      if (ok && nt > 0 && warp_wait(&pv_done[X], (nt - 1) & 1, &abort_flag, status)) {
+        tc_fence_after();
+        const float inv = 1.0f / l;
+        const bool row_ok = q0 + X * BQ + r < p.Lq;
+        bf16* O = (bf16*)p.out + (long long)(qrow0 + X * BQ + r) * p.ldo + h * HD;
 #pragma unroll 1
         for (int i = 0; i < HD / 32; ++i) {
           float t[32];
-          tmem_ld32(tmem + lane_off + C::O_COL + i * 32, t);
+          tmem_ld32(tO + i * 32, t);
+          if (row_ok) {
+            uint4* d4 = reinterpret_cast<uint4*>(O + i * 32);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) t[e] *= corr;
-          tmem_st32(tmem + lane_off + C::O_COL + i * 32, t);
-        }
-      }
-      l += sum;
-      m = m_use;
-      // P (bf16) row r into the K-major 128-byte-swizzled tile
-      uint8_t* P = smem + C::OFF_P + b * C::P_BYTES;
-#pragma unroll
-      for (int jj = 0; jj < 16; ++jj) {
-        uint32_t w[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          __nv_bfloat162 pr = __floats2bfloat162_rn(s[jj * 8 + 2 * e], s[jj * 8 + 2 * e + 1]);
-          w[e] = *reinterpret_cast<uint32_t*>(&pr);
-        }
-        const uint32_t off = (jj >> 3) * C::SUB_BYTES + r * 128 + ((((uint32_t)jj & 7u) ^ ((uint32_t)r & 7u)) << 4);
-        *reinterpret_cast<uint4*>(P + off) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      tc_fence_before();
-      mbar_arrive(&p_full[b]);
-    }
-    if (ok && nt > 0 &&
-        warp_wait(&pv_done[(nt - 1) & 1], ((nt - 1) >> 1) & 1, &abort_flag, status)) {
-      tc_fence_after();
-      const float inv = 1.0f / l;
-      const bool row_ok = qt * BQ + r < p.Lq;
-      bf16* O = (bf16*)p.out + (long long)(qrow0 + r) * p.ldo + h * HD;
-#pragma unroll 1
-      for (int i = 0; i < HD / 32; ++i) {
-        float t[32];
-        tmem_ld32(tmem + lane_off + C::O_COL + i * 32, t);
-        if (row_ok) {
-          uint4* d4 = reinterpret_cast<uint4*>(O + i * 32);
-#pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __nv_bfloat162 pr = __floats2bfloat162_rn(t[q4 * 8 + 2 * e] * inv, t[q4 * 8 + 2 * e + 1] * inv);
-              w[e] = *reinterpret_cast<uint32_t*>(&pr);
-            }
-            d4[q4] = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int q4 = 0; q4 < 4; ++q4)
+              d4[q4] = make_uint4(pack_bf16(t[q4 * 8] * inv, t[q4 * 8 + 1] * inv),
+                                  pack_bf16(t[q4 * 8 + 2] * inv, t[q4 * 8 + 3] * inv),
+                                  pack_bf16(t[q4 * 8 + 4] * inv, t[q4 * 8 + 5] * inv),
+                                  pack_bf16(t[q4 * 8 + 6] * inv, t[q4 * 8 + 7] * inv));
           }
         }
       }
@@ -356,9 +362,9 @@ cudaError_t launch(const AttnParams& p, int* status, cudaStream_t s) {
     maps.kp = maps.k;
     maps.vp = maps.v;
   }
-  dim3 grid((p.Lq + BQ - 1) / BQ, p.n_heads, p.n_chunks);
+  dim3 grid((p.Lq + 2 * BQ - 1) / (2 * BQ), p.n_heads, p.n_chunks);
   if (!status) status = op_status_word();
-  attn_tc_kernel<HD><<<grid, 192, C::SMEM, s>>>(maps, p, status);
+  attn_tc_kernel<HD><<<grid, 320, C::SMEM, s>>>(maps, p, status);
   return cudaGetLastError();
 }
 
