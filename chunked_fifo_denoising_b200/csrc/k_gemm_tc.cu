@@ -4,13 +4,15 @@
 // Euler scatter into the latent ring).
 //
 // Layout: 128 x BN output tiles, K in blocks of 64 (one 128-byte swizzled row
-// per operand row).  One CTA per SM, 6 warps:
+// per operand row).  One CTA per SM, 10 warps:
 //   warp 0      TMA producer (one thread): A and W tiles into a STAGES-deep ring
 //   warp 1      TMEM owner + MMA issuer (one thread): 4 x tcgen05.mma
 //               (M=128, N=BN, K=16) per k-block into one of two TMEM accumulators
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (thread = row),
-//               fused epilogue, 16-byte stores; frees the accumulator so the
-//               next tile's MMAs overlap this tile's epilogue.
+//   warps 2..9  epilogue, two warps per TMEM lane quarter (each half of the
+//               columns): tcgen05.ld of accumulator rows (thread = row), fused
+//               epilogue into a 128-byte-swizzled smem box, TMA store or TMA
+//               reduce-add; frees the accumulator so the next tile's MMAs
+//               overlap this tile's epilogue.
 // Tiles are walked row-block-major so the CTAs in flight share A row blocks
 // through L2 while W stays L2-resident.  Every mbarrier wait is bounded.
 #include <cstring>
@@ -86,12 +88,15 @@ struct GemmMaps {
 };
 
 template <int BN, int STAGES>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
 gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiParams e, int* status) {
   constexpr uint32_t A_BYTES = BM * BK * 2;
   constexpr uint32_t B_BYTES = BN * BK * 2;
   constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
-  constexpr uint32_t STG_OFF = STAGES * STAGE_BYTES;  // 4 warps x 2 staging boxes of 4 KB
+  constexpr uint32_t STG_OFF = STAGES * STAGE_BYTES;  // 8 warps x one 4 KB staging box
+  // columns per epilogue warp; with BN = 64 the second warp group has no columns
+  // and only keeps in step with the accumulator barriers
+  constexpr int HALF = BN >= 128 ? BN / 2 : BN;
   constexpr uint32_t TMEM_COLS = 2 * BN;
   constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, 0, 0);
 
@@ -114,7 +119,7 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull_bar[i], 1);
-      mbar_init(&tempty_bar[i], 128);
+      mbar_init(&tempty_bar[i], 256);
     }
     mbar_init(&done_bar, 1);
     abort_flag = 0;
@@ -202,10 +207,11 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
     }
     __syncwarp();
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
+    // ---------------- epilogue (warps 2..9) ----------------
+    // warps w and w+4 share TMEM lanes 32*(w%4).. and split the tile's columns
     const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31
-    uint8_t* stg = smem + STG_OFF + (warp - 2) * 8192;
-    uint32_t sb = 0;            // staging boxes used by this warp so far
+    const int half = (warp - 2) >> 2;
+    uint8_t* box = smem + STG_OFF + (warp - 2) * 4096;
     const bool bf16_out = (e.mode == EPI_STORE && !e.out_f32) || e.mode == EPI_GELU;
     const bool reduce = e.mode == EPI_RESID || e.mode == EPI_RESID_GATED;
     int it = 0;
@@ -216,13 +222,15 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
       const bool waited = mbar_wait(&tfull_bar[buf], acc_phase, &abort_flag, status, ST_TIMEOUT_GEMM);
       if (!__all_sync(0xffffffffu, waited)) break;
       tc_fence_after();
-      const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
+      const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN + half * HALF;
       const int row_base = m0 + quad * 32;
       const int row = row_base + lane;
-      const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN;
-      if (bf16_out) {
+      const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + half * HALF;
+      if (half * HALF >= BN) {
+        // no columns for this warp group
+      } else if (bf16_out) {
 #pragma unroll 1
-        for (int g = 0; g < BN / 64; ++g) {
+        for (int g = 0; g < HALF / 64; ++g) {
           const int col0 = n0 + g * 64;
           if (col0 >= N) break;  // uniform
           float v[64];
@@ -244,8 +252,7 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
             const int nchunk = min(8, (N - col0) / 8);
             for (int j = 0; j < nchunk; ++j) d[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
           }
-          uint8_t* box = stg + (sb & 1) * 4096;
-          if (lane == 0) bulk_wait_read<1>();  // the box written two rounds ago has been read
+          if (lane == 0) bulk_wait_read<0>();  // the previous store has read the box
           __syncwarp();
           stage_row(box, lane, w);
           fence_async_smem();
@@ -254,11 +261,10 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
             tma_store_2d(&maps.out, col0, row_base, box);
             bulk_commit();
           }
-          ++sb;
         }
       } else if (e.mode == EPI_EULER) {
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < HALF / 32; ++c) {
           float v[32];
           tmem_ld32(tbase + c * 32, v);
           const int col0 = n0 + c * 32;
@@ -278,7 +284,7 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
           gate = e.gate + sel * e.gate_stride;
         }
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = 0; c < HALF / 32; ++c) {
           const int col0 = n0 + c * 32;
           if (col0 >= N) break;  // uniform
           float v[32];
@@ -297,8 +303,7 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
           uint32_t w[32];
 #pragma unroll
           for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i]);
-          uint8_t* box = stg + (sb & 1) * 4096;
-          if (lane == 0) bulk_wait_read<1>();
+          if (lane == 0) bulk_wait_read<0>();
           __syncwarp();
           stage_row(box, lane, w);
           fence_async_smem();
@@ -308,7 +313,6 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
             else tma_store_2d(&maps.out, col0, row_base, box);
             bulk_commit();
           }
-          ++sb;
         }
       }
       tc_fence_before();
@@ -389,7 +393,7 @@ bool gemm_tc_supported(long long lda, int M, int N, int K) {
 template <int BN, int STAGES>
 static cudaError_t launch_tc(const bf16* A, long long lda, const bf16* W, int M, int N, int K,
                              const EpiParams& e, int* status, cudaStream_t s) {
-  constexpr int SMEM = STAGES * (BM * BK * 2 + BN * BK * 2) + 4 * 8192 + 1024;
+  constexpr int SMEM = STAGES * (BM * BK * 2 + BN * BK * 2) + 8 * 4096 + 1024;
   static std::once_flag once;
   static cudaError_t attr_err = cudaSuccess;
   std::call_once(once, [] {
@@ -413,7 +417,7 @@ static cudaError_t launch_tc(const bf16* A, long long lda, const bf16* W, int M,
   const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
   const int grid = tiles < sm_count() ? tiles : sm_count();
   if (!status) status = op_status_word();
-  gemm_tc_kernel<BN, STAGES><<<grid, 192, SMEM, s>>>(maps, M, N, K, e, status);
+  gemm_tc_kernel<BN, STAGES><<<grid, 320, SMEM, s>>>(maps, M, N, K, e, status);
   return cudaGetLastError();
 }
 

@@ -96,10 +96,91 @@ __global__ void __launch_bounds__(LN_THREADS) ln_mod_kernel(LnParams p) {
   }
 }
 
+// One warp per row for narrow rows (d <= 512), where a 128-thread block per
+// row would leave most threads idle: both reductions are warp shuffles, 8 rows
+// per 256-thread block.
+constexpr int LNW_MAXV = 16;
+
+template <bool OUT_F32>
+__global__ void __launch_bounds__(256) ln_mod_warp_kernel(LnParams p) {
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= p.M) return;
+  const int nv = p.d >> 2;
+  const float4* xr = reinterpret_cast<const float4*>(p.x + (long long)row * p.ldx);
+  float4 v[LNW_MAXV];
+  float s = 0.0f;
+#pragma unroll
+  for (int i = 0; i < LNW_MAXV; ++i) {
+    const int idx = lane + i * 32;
+    if (idx < nv) {
+      v[i] = xr[idx];
+      s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+  const float mean = s / (float)p.d;
+  float ss = 0.0f;
+#pragma unroll
+  for (int i = 0; i < LNW_MAXV; ++i) {
+    const int idx = lane + i * 32;
+    if (idx < nv) {
+      const float a = v[i].x - mean, b = v[i].y - mean, c = v[i].z - mean, d = v[i].w - mean;
+      ss += (a * a + b * b) + (c * c + d * d);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float rstd = 1.0f / sqrtf(ss / (float)p.d + 1e-6f);
+  const float4* sh = nullptr;
+  const float4* sc = nullptr;
+  if (p.shift) {
+    const int c = row / p.rows_per_chunk;
+    const long long sel = p.chunk_sel ? p.chunk_sel[c] : c;
+    sh = reinterpret_cast<const float4*>(p.shift + sel * p.mod_stride);
+    sc = reinterpret_cast<const float4*>(p.scale + sel * p.mod_stride);
+  }
+#pragma unroll
+  for (int i = 0; i < LNW_MAXV; ++i) {
+    const int idx = lane + i * 32;
+    if (idx < nv) {
+      float4 o;
+      o.x = (v[i].x - mean) * rstd;
+      o.y = (v[i].y - mean) * rstd;
+      o.z = (v[i].z - mean) * rstd;
+      o.w = (v[i].w - mean) * rstd;
+      if (sh) {
+        const float4 a = sh[idx], b = sc[idx];
+        o.x = o.x * (1.0f + b.x) + a.x;
+        o.y = o.y * (1.0f + b.y) + a.y;
+        o.z = o.z * (1.0f + b.z) + a.z;
+        o.w = o.w * (1.0f + b.w) + a.w;
+      }
+      if (OUT_F32) {
+        reinterpret_cast<float4*>((float*)p.out + (long long)row * p.ldo)[idx] = o;
+      } else {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(o.z, o.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        reinterpret_cast<uint2*>((bf16*)p.out + (long long)row * p.ldo)[idx] = pk;
+      }
+    }
+  }
+}
+
 cudaError_t layernorm_mod(const LnParams& p, cudaStream_t s) {
   if (p.M <= 0) return cudaSuccess;
-  if (p.out_f32) ln_mod_kernel<true><<<p.M, LN_THREADS, 0, s>>>(p);
-  else ln_mod_kernel<false><<<p.M, LN_THREADS, 0, s>>>(p);
+  if (p.d <= 512) {
+    const int blocks = (p.M + 7) / 8;
+    if (p.out_f32) ln_mod_warp_kernel<true><<<blocks, 256, 0, s>>>(p);
+    else ln_mod_warp_kernel<false><<<blocks, 256, 0, s>>>(p);
+  } else {
+    if (p.out_f32) ln_mod_kernel<true><<<p.M, LN_THREADS, 0, s>>>(p);
+    else ln_mod_kernel<false><<<p.M, LN_THREADS, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 

@@ -69,6 +69,7 @@ def run_gemm(A, W, bias, epi, out=None, resid=None, gate=None, sel=None, rpc=1, 
 
 
 @pytest.mark.parametrize("M,N,K", [(300, 256, 128), (129, 64, 64), (1000, 384, 192),
+                                   (300, 192, 128), (200, 96, 64),
                                    (2048, 1536, 512), (257, 4608, 1536)])
 def test_gemm_store_bf16(M, N, K):
     A, W = gen((M, K), seed=1), gen((N, K), 0.02, seed=2)
