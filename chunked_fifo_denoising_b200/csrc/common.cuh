@@ -18,6 +18,37 @@ __device__ __forceinline__ float gelu_erf(float x) {
 }
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
 
+// GELU x * Phi(x) with erf from Abramowitz and Stegun, Handbook of
+// Mathematical Functions, formula 7.1.26 (|error of erf| <= 1.5e-7):
+// erf(z) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2),
+// t = 1 / (1 + p z), z >= 0; erf is odd.  Branch-free, used by the
+// tensor-core GEMM epilogue; the reciprocal and 2^x run on the MUFU unit
+// (approximate, relative error ~1e-7, well inside the formula's bound).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+__device__ __forceinline__ float ex2_approx_f(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float gelu_as(float x) {
+  const float z = fabsf(x) * 0.70710678118654752f;
+  const float t = rcp_approx(fmaf(0.3275911f, z, 1.0f));
+  float poly = fmaf(1.061405429f, t, -1.453152027f);
+  poly = fmaf(poly, t, 1.421413741f);
+  poly = fmaf(poly, t, -0.284496736f);
+  poly = fmaf(poly, t, 0.254829592f);
+  poly *= t;
+  const float e = ex2_approx_f(-z * z * 1.4426950408889634f);
+  const float erf_abs = fmaf(-poly, e, 1.0f);
+  const float erf_x = copysignf(erf_abs, x);
+  return 0.5f * x * (1.0f + erf_x);
+}
+
 // Ring offset of (row, col) of the head output: row = token of batch chunk,
 // col = patch feature.  Inverse of the patch gather.
 __device__ __forceinline__ long long euler_index(const EpiParams& e, int row, int col, int Lc) {

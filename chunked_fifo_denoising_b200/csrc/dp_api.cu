@@ -719,6 +719,12 @@ dp_status dp_queue_init(dp_model* m, const dp_queue_config* qc, const float* tex
   for (int i = 0; i < DP_PARAM_COUNT; ++i)
     for (char sset : m->params[i].set)
       if (!sset) return fail(DP_ERR_STATE, "parameter %d not set", i);
+  {
+    // kernels index rows with 32-bit integers and elements with 64-bit offsets
+    const long long lc = (long long)(qc->frames_per_chunk / c.patch_t) * (qc->lat_h / c.patch_h) *
+                         (qc->lat_w / c.patch_w);
+    if ((long long)qc->T * lc >= (1LL << 31)) return fail(DP_ERR_INVALID_ARG, "too many rows for one queue step");
+  }
   dp_queue* q = new dp_queue();
   q->m = m;
   q->qc = *qc;
@@ -730,8 +736,6 @@ dp_status dp_queue_init(dp_model* m, const dp_queue_config* qc, const float* tex
   const int d = m->d, L = m->L;
   const size_t as = m->act_size();
   const long long Mm = q->Mmax;
-  if (Mm * (long long)std::max(3 * d, m->F) >= (1LL << 31) * 2)
-    return fail(DP_ERR_INVALID_ARG, "activation buffers exceed the 32-bit row index range");
   dp_status s = DP_OK;
 #define QA(buf, bytes, what) if (s == DP_OK) s = dev_alloc(buf, bytes, what)
   QA(q->ring, (size_t)q->n_slots * q->chunk_numel * 4, "latent ring");

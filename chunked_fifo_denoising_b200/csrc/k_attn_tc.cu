@@ -260,31 +260,45 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
         tc_fence_after();
         float s[128];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) tmem_ld32(tS + i * 32, *reinterpret_cast<float(*)[32]>(s + i * 32));
+        for (int i = 0; i < 4; ++i) tmem_ld32_nowait(tS + i * 32, *reinterpret_cast<float(*)[32]>(s + i * 32));
+        tmem_wait_ld();
         const int valid = tile_valid(j, tiles_p, n_p, n_o);
         if (valid < BKV) {
 #pragma unroll
           for (int i = 0; i < 128; ++i)
             if (i >= valid) s[i] = -INFINITY;
         }
-        float mx = s[0];
+        // row maximum with 8 independent partial maxima (short dependency chains)
+        float mxp[8];
 #pragma unroll
-        for (int i = 1; i < 128; ++i) mx = fmaxf(mx, s[i]);
+        for (int i = 0; i < 8; ++i) mxp[i] = s[i];
+#pragma unroll
+        for (int i = 8; i < 128; ++i) mxp[i & 7] = fmaxf(mxp[i & 7], s[i]);
+        const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                               fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
         const float m_new = fmaxf(m, mx * sl2);
         const bool want = (m == -INFINITY) || (m_new > m + 8.0f);
         const bool resc = __any_sync(0xffffffffu, want);  // TMEM access is warp-collective
         const float m_use = resc ? m_new : m;
         const float nm = -m_use;
-        float sum0 = 0.0f, sum1 = 0.0f;
-        uint32_t w[64];
+        float sp[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+        // P (bf16, two keys per 32-bit column) over the first 64 columns of S, 32
+        // keys at a time; S is already in registers, and PV of the previous tile
+        // (which read the old P) completed before S of this tile was written
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float a = ex2_approx(fmaf(s[2 * i], sl2, nm));
-          const float b = ex2_approx(fmaf(s[2 * i + 1], sl2, nm));
-          sum0 += a;
-          sum1 += b;
-          w[i] = pack_bf16(a, b);
+        for (int q = 0; q < 4; ++q) {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a = ex2_approx(fmaf(s[32 * q + 2 * i], sl2, nm));
+            const float b = ex2_approx(fmaf(s[32 * q + 2 * i + 1], sl2, nm));
+            sp[(2 * i) & 7] += a;
+            sp[(2 * i + 1) & 7] += b;
+            w[i] = pack_bf16(a, b);
+          }
+          tmem_st16_nowait(tS + q * 16, w);
         }
+        tmem_wait_st();
         if (resc && j > 0) {
           // O must hold PV of every earlier tile before it is rescaled
           if (!warp_wait(&pv_done[X], (j - 1) & 1, &abort_flag, status)) { ok = false; break; }
@@ -300,12 +314,8 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
             tmem_st32(tO + i * 32, t);
           }
         }
-        l += sum0 + sum1;
+        l += ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
         m = m_use;
-        // P (bf16, two keys per column) over the first 64 columns of S
-#pragma unroll
-        for (int i = 0; i < 4; ++i) tmem_st16_nowait(tS + i * 16, w + i * 16);
-        tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[X]);
       }

@@ -240,7 +240,7 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
           add_bias<64>(e, col0, N, v);
           if (e.mode == EPI_GELU) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] = gelu_erf(v[i]);
+            for (int i = 0; i < 64; ++i) v[i] = gelu_as(v[i]);
           }
           uint32_t w[32];
 #pragma unroll
@@ -287,17 +287,22 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
         for (int c = 0; c < HALF / 32; ++c) {
           const int col0 = n0 + c * 32;
           if (col0 >= N) break;  // uniform
+          // gate loads first: their latency overlaps the TMEM load
+          float4 gg[8];
+          if (gate) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) gg[i] = reinterpret_cast<const float4*>(gate + col0)[i];
+          }
           float v[32];
           tmem_ld32(tbase + c * 32, v);
           add_bias<32>(e, col0, N, v);
           if (gate) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              const float4 gg = reinterpret_cast<const float4*>(gate + col0)[i];
-              v[4 * i] *= gg.x;
-              v[4 * i + 1] *= gg.y;
-              v[4 * i + 2] *= gg.z;
-              v[4 * i + 3] *= gg.w;
+              v[4 * i] *= gg[i].x;
+              v[4 * i + 1] *= gg[i].y;
+              v[4 * i + 2] *= gg[i].z;
+              v[4 * i + 3] *= gg[i].w;
             }
           }
           uint32_t w[32];

@@ -171,9 +171,101 @@ __global__ void __launch_bounds__(256) ln_mod_warp_kernel(LnParams p) {
   }
 }
 
+// Rows of d = 512 * NV: 8 consecutive rows per 128-thread block; the loads of
+// row i+1 are issued before the reductions of row i, so every thread keeps
+// 2 * NV 16-byte loads in flight.
+constexpr int LN_ROWS = 8;
+
+template <int NV, bool OUT_F32>
+__global__ void __launch_bounds__(LN_THREADS) ln_rows_kernel(LnParams p) {
+  __shared__ float red[2][LN_THREADS / 32];
+  const int row0 = blockIdx.x * LN_ROWS;
+  const int rend = min(row0 + LN_ROWS, p.M);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  float4 v[NV], nx[NV];
+  auto load = [&](float4 (&dst)[NV], int row) {
+    const float4* xr = reinterpret_cast<const float4*>(p.x + (long long)row * p.ldx);
+#pragma unroll
+    for (int i = 0; i < NV; ++i) dst[i] = xr[threadIdx.x + i * LN_THREADS];
+  };
+  auto reduce = [&](float a, int b) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a += __shfl_xor_sync(0xffffffffu, a, o);
+    if (lane == 0) red[b][wid] = a;
+    __syncthreads();
+    float t = 0.0f;
+#pragma unroll
+    for (int i = 0; i < LN_THREADS / 32; ++i) t += red[b][i];
+    return t;
+  };
+  if (row0 < rend) load(v, row0);
+  for (int row = row0; row < rend; ++row) {
+    if (row + 1 < rend) load(nx, row + 1);
+    float s = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) s += (v[i].x + v[i].y) + (v[i].z + v[i].w);
+    const float mean = reduce(s, 0) / (float)p.d;
+    float ss = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const float a = v[i].x - mean, b = v[i].y - mean, c = v[i].z - mean, d = v[i].w - mean;
+      ss += (a * a + b * b) + (c * c + d * d);
+    }
+    const float var = reduce(ss, 1) / (float)p.d;
+    const float rstd = 1.0f / sqrtf(var + 1e-6f);
+    const float4* sh = nullptr;
+    const float4* sc = nullptr;
+    if (p.shift) {
+      const int c = row / p.rows_per_chunk;
+      const long long sel = p.chunk_sel ? p.chunk_sel[c] : c;
+      sh = reinterpret_cast<const float4*>(p.shift + sel * p.mod_stride);
+      sc = reinterpret_cast<const float4*>(p.scale + sel * p.mod_stride);
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      const int idx = threadIdx.x + i * LN_THREADS;
+      float4 o;
+      o.x = (v[i].x - mean) * rstd;
+      o.y = (v[i].y - mean) * rstd;
+      o.z = (v[i].z - mean) * rstd;
+      o.w = (v[i].w - mean) * rstd;
+      if (sh) {
+        const float4 a = sh[idx], b = sc[idx];
+        o.x = o.x * (1.0f + b.x) + a.x;
+        o.y = o.y * (1.0f + b.y) + a.y;
+        o.z = o.z * (1.0f + b.z) + a.z;
+        o.w = o.w * (1.0f + b.w) + a.w;
+      }
+      if (OUT_F32) {
+        reinterpret_cast<float4*>((float*)p.out + (long long)row * p.ldo)[idx] = o;
+      } else {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(o.x, o.y);
+        __nv_bfloat162 hi = __floats2bfloat162_rn(o.z, o.w);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t*>(&lo);
+        pk.y = *reinterpret_cast<uint32_t*>(&hi);
+        reinterpret_cast<uint2*>((bf16*)p.out + (long long)row * p.ldo)[idx] = pk;
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) v[i] = nx[i];
+  }
+}
+
+template <int NV>
+static void launch_rows(const LnParams& p, cudaStream_t s) {
+  const int blocks = (p.M + LN_ROWS - 1) / LN_ROWS;
+  if (p.out_f32) ln_rows_kernel<NV, true><<<blocks, LN_THREADS, 0, s>>>(p);
+  else ln_rows_kernel<NV, false><<<blocks, LN_THREADS, 0, s>>>(p);
+}
+
 cudaError_t layernorm_mod(const LnParams& p, cudaStream_t s) {
   if (p.M <= 0) return cudaSuccess;
-  if (p.d <= 512) {
+  if (p.d == 1536) {
+    launch_rows<3>(p, s);
+  } else if (p.d == 5120) {
+    launch_rows<10>(p, s);
+  } else if (p.d <= 512) {
     const int blocks = (p.M + 7) / 8;
     if (p.out_f32) ln_mod_warp_kernel<true><<<blocks, 256, 0, s>>>(p);
     else ln_mod_warp_kernel<false><<<blocks, 256, 0, s>>>(p);

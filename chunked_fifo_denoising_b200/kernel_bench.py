@@ -31,18 +31,71 @@ CASES = {
 }
 
 
+class _ClockSampler:
+    """Median SM clock (MHz) over a timed loop, read through NVML in a thread."""
+
+    def __init__(self):
+        import threading
+        self.samples = []
+        self.stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(torch.cuda.current_device())
+            self.nv = pynvml
+        except Exception:
+            self.nv = None
+        self.t = threading.Thread(target=self._run, daemon=True)
+
+    def _run(self):
+        while not self.stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+            except Exception:
+                return
+            self.stop.wait(0.005)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self.stop.set()
+        if self.nv is not None:
+            self.t.join()
+
+    def median(self):
+        s = sorted(self.samples)
+        return float(s[len(s) // 2]) if s else None
+
+
 def _time(fn, iters, stream):
+    """Mean ms per launch and the median SM clock (MHz) while timing."""
     for _ in range(2):
         fn()
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(iters):
-        fn()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    return e0.elapsed_time(e1) / iters
+    with _ClockSampler() as ck:
+        e0.record(stream)
+        for _ in range(iters):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / iters, ck.median()
+
+
+def _res(d, ms, mhz, tflops=None, gbs=None):
+    d["ms"] = ms
+    d["sm_mhz"] = mhz
+    if tflops is not None:
+        d["tflops"] = tflops
+        if mhz:  # the same work at the 1965 MHz maximum clock, for comparing runs
+            d["tflops_at_max_clock"] = tflops * 1965.0 / mhz
+    if gbs is not None:
+        d["gbs"] = gbs
+    return d
 
 
 def run_case(name, iters, chunks):
@@ -73,9 +126,9 @@ def run_case(name, iters, chunks):
 
         def fn():
             B.check(B.dp_op_gemm(a, sh), "dp_op_gemm")
-        ms = _time(fn, iters, stream)
+        ms, mhz = _time(fn, iters, stream)
         B.check(B.dp_op_check(sh), "dp_op_check")
-        return {"case": name, "M": M, "N": N, "K": K, "ms": ms, "tflops": 2.0 * M * N * K / ms / 1e9}
+        return _res({"case": name, "M": M, "N": N, "K": K}, ms, mhz, tflops=2.0 * M * N * K / ms / 1e9)
     if kind == "attn":
         H, hd, Lk, shared = c["H"], c["hd"], c["Lk"], c["shared"]
         d = H * hd
@@ -102,10 +155,10 @@ def run_case(name, iters, chunks):
 
         def fn():
             B.check(B.dp_op_attention(a, sh), "dp_op_attention")
-        ms = _time(fn, iters, stream)
+        ms, mhz = _time(fn, iters, stream)
         B.check(B.dp_op_check(sh), "dp_op_check")
         flops = 4.0 * Lc * keys * d
-        return {"case": name, "chunks": chunks, "Lq": Lc, "heads": H, "ms": ms, "tflops": flops / ms / 1e9}
+        return _res({"case": name, "chunks": chunks, "Lq": Lc, "heads": H}, ms, mhz, tflops=flops / ms / 1e9)
     if kind == "ln":
         d = c["d"]
         x = torch.randn(M, d, device="cuda", generator=g)
@@ -118,8 +171,8 @@ def run_case(name, iters, chunks):
 
         def fn():
             B.check(B.dp_op_layernorm_mod(a, sh), "dp_op_layernorm_mod")
-        ms = _time(fn, iters, stream)
-        return {"case": name, "M": M, "d": d, "ms": ms, "gbs": M * d * 6.0 / ms / 1e6}
+        ms, mhz = _time(fn, iters, stream)
+        return _res({"case": name, "M": M, "d": d}, ms, mhz, gbs=M * d * 6.0 / ms / 1e6)
     raise ValueError(name)
 
 

@@ -244,12 +244,24 @@ def test_self_attention_full_size_sampled_rows():
         assert rel_l2(f64(out[sl][rows]), ref) < 1e-2, c
 
 
+def test_cross_attention_full_size_sampled_rows():
+    """Wan-1.3B: 156 000 queries against the 512 prompt keys of one layer."""
+    n, Lc, H, hd, Lt = 50, 3120, 12, 128, 512
+    d = H * hd
+    q = gen((n * Lc, d), 1.0, torch.bfloat16, seed=60)
+    kv = gen((Lt, 2 * d), 1.0, torch.bfloat16, seed=61)
+    out = run_attn(q, kv[:, :d], kv[:, d:], n, Lc, H, hd, Lt, 0, 0)
+    rows = np.unique(np.concatenate([np.random.default_rng(1).integers(0, n * Lc, 40), [0, n * Lc - 1]]))
+    ref = dit.attention(f64(q[rows]), f64(kv[:, :d]), f64(kv[:, d:]), H)
+    assert rel_l2(f64(out[rows]), ref) < 1e-2
+
+
 # ---------------------------------------------------------------------------
 # layer norm + modulation
 # ---------------------------------------------------------------------------
 
 @pytest.mark.parametrize("out_dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("M,d", [(1000, 1536), (33, 64), (257, 5120)])
+@pytest.mark.parametrize("M,d", [(1000, 1536), (33, 64), (257, 5120), (333, 512), (156000, 1536)])
 def test_layernorm_mod(out_dtype, M, d):
     x = gen((M, d), 2.0, torch.float32, seed=50) + 0.5
     table = gen((5, 2 * d), 0.3, torch.float32, seed=51)

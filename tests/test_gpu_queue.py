@@ -7,7 +7,9 @@ float64 oracle on identical seeded inputs:
   exactly equal to the oracle queue on the (T, N) schedule of every workload;
 * bf16 production mode: one queue step from the same state within relative L2
   2e-2 on the velocity of every chunk, on the persisted K/V and on the latents
-  (small workload; Wan-1.3B shapes with two layers);
+  (small workload; Wan-1.3B shapes with two layers; Wan-14B shapes with one
+  layer);
+* resuming from latents and persisted K/V read mid-stream is bit-exact;
 * error codes, the internal noise generator, flat device memory.
 """
 import numpy as np
@@ -111,44 +113,44 @@ def test_bookkeeping_exact_on_every_schedule(name):
     model.close()
 
 
-def _one_step_parity(w, n_layers=None, seed_state=7):
-    """Queue state just before a step: chunks at levels 1, 2, 3 (no push), the
-    head's predecessor K/V persisted; compare one GPU step with the oracle."""
+def _one_step_parity(w, n_layers=None, n_occ=3, seed_state=7):
+    """Queue state just before a step: chunks at levels 1 .. n_occ (no push),
+    the head's predecessor K/V persisted; compare one GPU step with the oracle."""
     if n_layers is not None:
         w = synth.truncated(w, n_layers)
     m, q = w.model, w.queue
     T = q.T
     n_chunks = 20
-    step = n_chunks + T - 4          # chunks 17, 18, 19 at levels 1, 2, 3
-    head = n_chunks - 3
+    head = n_chunks - n_occ
+    step = head + T - 1              # the head chunk is at level 1
     model, queue, p, text = make(w, "bf16", n_chunks=n_chunks)
     rng = np.random.default_rng(seed_state)
-    lat = rng.standard_normal((3,) + q.chunk_shape(m)).astype(np.float32)
+    lat = rng.standard_normal((n_occ,) + q.chunk_shape(m)).astype(np.float32)
     Lc = q.tokens_per_chunk(m)
     kv = bf16_round(rng.standard_normal((m.n_layers, 2, Lc, m.dim)).astype(np.float32) * 0.5)
     queue.load_state(step, n_chunks, lat, kv)
     info = queue.inspect()
-    assert info["ids"] == [head, head + 1, head + 2] and info["levels"] == [1, 2, 3]
+    assert info["ids"] == list(range(head, n_chunks)) and info["levels"] == list(range(1, n_occ + 1))
     assert info["head_pred"] == 2 and info["writes_cache"] == 1
     queue.step(None)
     queue.sync()
     popped = np.empty(q.chunk_shape(m), np.float32)
     assert queue.pop(popped) == head
-    rest = queue.read_latents(2)
+    rest = queue.read_latents(n_occ - 1)
     new_kv, kv_id = queue.read_pred_kv()
     assert kv_id == head
     # oracle
     fn = dit.make_velocity_fn(p, text, m, T)
     st = fifo.QueueState(T=T, n_chunks=n_chunks, step=step, next_id=n_chunks,
-                         entries=[fifo.Entry(head + i, 1 + i, lat[i].astype(np.float64)) for i in range(3)],
+                         entries=[fifo.Entry(head + i, 1 + i, lat[i].astype(np.float64)) for i in range(n_occ)],
                          pred_id=head - 1, pred_kv=[(kv[l, 0], kv[l, 1]) for l in range(m.n_layers)])
     tr = fifo.queue_step(st, fn, None)
     assert tr.popped == [head]
     ref_pop = st.ready[0][1]
     ref_rest = [e.latent for e in st.entries]
     dsig = -1.0 / T
-    v_gpu = [(popped - lat[0]) / dsig] + [(rest[i] - lat[i + 1]) / dsig for i in range(2)]
-    v_ref = [(ref_pop - lat[0]) / dsig] + [(ref_rest[i] - lat[i + 1]) / dsig for i in range(2)]
+    v_gpu = [(popped - lat[0]) / dsig] + [(rest[i] - lat[i + 1]) / dsig for i in range(n_occ - 1)]
+    v_ref = [(ref_pop - lat[0]) / dsig] + [(ref_rest[i] - lat[i + 1]) / dsig for i in range(n_occ - 1)]
     errs = [rel_l2(a, b) for a, b in zip(v_gpu, v_ref)]
     assert max(errs) <= 2e-2, errs
     assert rel_l2(popped, ref_pop) <= 2e-2
@@ -165,6 +167,51 @@ def test_bf16_step_small():
 
 def test_bf16_step_wan13b_shapes_two_layers():
     _one_step_parity(synth.WORKLOADS["wan1.3b_480p"], n_layers=2)
+
+
+def test_bf16_step_wan14b_shapes_one_layer():
+    """Wan-14B shapes (d 5120, 40 heads, 7200 tokens per chunk), one layer, the
+    head chunk alone with its persisted predecessor."""
+    _one_step_parity(synth.WORKLOADS["wan14b_720p"], n_layers=1, n_occ=1)
+
+
+def test_checkpoint_resume_is_bit_exact():
+    """Latents and persisted K/V read mid-stream and loaded into a new queue
+    continue the stream with bit-identical outputs."""
+    from chunked_fifo_denoising_b200 import Queue
+    w = synth.truncated(synth.WORKLOADS["small_bf16"], 2)
+    m, q = w.model, w.queue
+    N, s_ck = 14, 12
+    model, qa, p, text = make(w, "bf16", n_chunks=N)
+    out = np.empty(q.chunk_shape(m), np.float32)
+    got_a, got_b = {}, {}
+    for _ in range(s_ck):
+        qa.step(None)
+        while qa.try_pop(out)[0] == 0:
+            pass
+    info = qa.inspect()
+    n_q = info["n"] - (1 if info["next_push_id"] >= 0 else 0)
+    lat = qa.read_latents(n_q)
+    kv, kv_id = qa.read_pred_kv()
+    n_pushed = info["next_push_id"] if info["next_push_id"] >= 0 else N
+    qb = Queue(model, text, q.T, q.frames_per_chunk, q.lat_h, q.lat_w, N)
+    qb.load_state(info["step"], n_pushed, lat, kv if kv_id >= 0 else None)
+    for qq, got in ((qa, got_a), (qb, got_b)):
+        while qq.try_step(None) == 0:
+            while True:
+                st, cid = qq.try_pop(out)
+                if st != 0:
+                    break
+                got[cid] = out.copy()
+        while True:
+            st, cid = qq.try_pop(out)
+            if st != 0:
+                break
+            got[cid] = out.copy()
+    assert sorted(got_a) == sorted(got_b) and len(got_a) > 0
+    for k in got_a:
+        assert np.array_equal(got_a[k], got_b[k]), k
+    model.close()
 
 
 def test_errors_full_empty_drained():
