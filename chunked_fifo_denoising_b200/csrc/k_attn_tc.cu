@@ -66,6 +66,32 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, w);
 }
 
+// Packed fp32x2 arithmetic of sm_100 (two lanes per instruction, each lane
+// rounded as the scalar instruction) and the three-input maximum.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -273,15 +299,16 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
 #pragma unroll
         for (int i = 0; i < 8; ++i) mxp[i] = s[i];
 #pragma unroll
-        for (int i = 8; i < 128; ++i) mxp[i & 7] = fmaxf(mxp[i & 7], s[i]);
-        const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                               fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+        for (int i = 8; i < 128; i += 2) mxp[(i >> 1) & 7] = max3f(mxp[(i >> 1) & 7], s[i], s[i + 1]);
+        const float mx = fmaxf(max3f(mxp[0], mxp[1], mxp[2]),
+                               fmaxf(max3f(mxp[3], mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
         const float m_new = fmaxf(m, mx * sl2);
         const bool want = (m == -INFINITY) || (m_new > m + 8.0f);
         const bool resc = __any_sync(0xffffffffu, want);  // TMEM access is warp-collective
         const float m_use = resc ? m_new : m;
         const float nm = -m_use;
-        float sp[8] = {0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f, 0.0f};
+        const uint64_t sl2x2 = f2_pack(sl2, sl2), nmx2 = f2_pack(nm, nm);
+        uint64_t sp2[4] = {0ull, 0ull, 0ull, 0ull};  // packed partial row sums
         // P (bf16, two keys per 32-bit column) over the first 64 columns of S, 32
         // keys at a time; S is already in registers, and PV of the previous tile
         // (which read the old P) completed before S of this tile was written
@@ -290,10 +317,11 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float a = ex2_approx(fmaf(s[32 * q + 2 * i], sl2, nm));
-            const float b = ex2_approx(fmaf(s[32 * q + 2 * i + 1], sl2, nm));
-            sp[(2 * i) & 7] += a;
-            sp[(2 * i + 1) & 7] += b;
+            float xa, xb;
+            f2_unpack(f2_fma(f2_pack(s[32 * q + 2 * i], s[32 * q + 2 * i + 1]), sl2x2, nmx2), xa, xb);
+            const float a = ex2_approx(xa);
+            const float b = ex2_approx(xb);
+            sp2[i & 3] = f2_add(sp2[i & 3], f2_pack(a, b));
             w[i] = pack_bf16(a, b);
           }
           tmem_st16_nowait(tS + q * 16, w);
@@ -314,7 +342,13 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
             tmem_st32(tO + i * 32, t);
           }
         }
-        l += ((sp[0] + sp[1]) + (sp[2] + sp[3])) + ((sp[4] + sp[5]) + (sp[6] + sp[7]));
+        {
+          float t0, t1, t2, t3;
+          f2_unpack(f2_add(f2_add(sp2[0], sp2[1]), f2_add(sp2[2], sp2[3])), t0, t1);
+          (void)t2;
+          (void)t3;
+          l += t0 + t1;
+        }
         m = m_use;
         tc_fence_before();
         mbar_arrive(&p_full[X]);
