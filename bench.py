@@ -68,15 +68,19 @@ def gemm_traffic():
     return int(m.group(1))
 
 
-def step_flops(m, q, occ):
+def step_flops(m, q, occ, neighbours="pred"):
     """Algorithmic FLOPs of one step with `occ` queued chunks, every chunk with
     a full predecessor: per token per layer 12 d^2 + 4 d F + 4 (2 Lc) d + 4 Lt d,
-    plus the patch and head projections (2 * 64 * d each per token)."""
+    plus the patch and head projections (2 * 64 * d each per token).  With the
+    successor link, every chunk but the last also reads Lc more keys."""
     Lc = q.tokens_per_chunk(m)
     d, F = m.dim, m.ffn_dim
     per_tok_layer = 12 * d * d + 4 * d * F + 4 * (2 * Lc) * d + 4 * m.text_len * d
     toks = occ * Lc
-    return toks * (m.n_layers * per_tok_layer + 2 * 2 * m.patch_dim * d)
+    flops = toks * (m.n_layers * per_tok_layer + 2 * 2 * m.patch_dim * d)
+    if neighbours == "both":
+        flops += m.n_layers * 4.0 * Lc * ((occ - 1) * Lc) * d
+    return flops
 
 
 class Clocks:
@@ -250,7 +254,7 @@ def run_ours(args, w):
     # random-init weights on the device, N(0, 0.02^2), seeded per rank
     g = torch.Generator(device="cuda").manual_seed(1000 + rank)
     import synth
-    model = Model(m, "bf16", stream=stream)
+    model = Model(m, "bf16", stream=stream, neighbours=args.neighbours)
     for name, shape, per_layer in synth.param_specs(m):
         for l in range(m.n_layers if per_layer else 1):
             t = torch.randn(shape, generator=g, device="cuda") * 0.02
@@ -313,7 +317,7 @@ def run_ours(args, w):
     value = whole_job_rate(world, args.steps, frames, ms)
     e2e_value = whole_job_rate(world, args.e2e_steps, frames, ms_e2e)
     pk = peaks()
-    flops = step_flops(m, q, occ)
+    flops = step_flops(m, q, occ, args.neighbours)
     ms_step = ms / args.steps
     peak_tf = pk["bf16_tflops_sustained"]
     gemm = kt["gemm"]
@@ -333,7 +337,8 @@ def run_ours(args, w):
             "config": {"workload": w.name, "T": T, "occupancy": occ, "chunk_tokens": q.tokens_per_chunk(m),
                        "tokens_per_step": occ * q.tokens_per_chunk(m), "frames_per_step": frames,
                        "layers": m.n_layers, "dim": m.dim, "ffn": m.ffn_dim, "heads": m.n_heads,
-                       "text_tokens": m.text_len, "parallelism": f"replicas x{world}",
+                       "text_tokens": m.text_len, "neighbours": args.neighbours,
+                       "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (fp32 residual stream alone is "
                              f"{occ * q.tokens_per_chunk(m) * m.dim * 4 / 1e6:.0f} MB)"},
             "pct_bf16_peak": 100.0 * flops / (ms_step / 1e3) / (peak_tf * 1e12),
@@ -370,6 +375,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="wan1.3b_480p")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--neighbours", default="pred", choices=["pred", "both"],
+                    help="self-attention neighbourhood: predecessor only, or also the successor")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -18,6 +18,7 @@ STATUS_NAMES = ["DP_OK", "DP_ERR_INVALID_ARG", "DP_ERR_OOM", "DP_ERR_CUDA", "DP_
                 "DP_ERR_FULL", "DP_ERR_DRAINED", "DP_ERR_STATE", "DP_ERR_KERNEL"]
 DP_PREC_BF16, DP_PREC_FP32_VALIDATE = 0, 1
 DP_LOC_DEVICE, DP_LOC_HOST = 0, 1
+DP_NEIGHBOURS_PRED, DP_NEIGHBOURS_BOTH = 0, 1
 DP_DT_F32, DP_DT_BF16 = 0, 1
 DP_EPI_STORE, DP_EPI_GELU, DP_EPI_RESID, DP_EPI_RESID_GATED = 0, 1, 2, 3
 DP_KCLASS_COUNT = 7
@@ -40,7 +41,8 @@ class dp_model_config(C.Structure):
     _fields_ = [("n_layers", C.c_int), ("dim", C.c_int), ("n_heads", C.c_int),
                 ("ffn_dim", C.c_int), ("freq_dim", C.c_int), ("latent_ch", C.c_int),
                 ("patch_t", C.c_int), ("patch_h", C.c_int), ("patch_w", C.c_int),
-                ("text_len", C.c_int), ("text_in_dim", C.c_int), ("prec", C.c_int)]
+                ("text_len", C.c_int), ("text_in_dim", C.c_int), ("prec", C.c_int),
+                ("neighbours", C.c_int)]
 
 
 class dp_queue_config(C.Structure):
@@ -71,7 +73,8 @@ class dp_attn_args(C.Structure):
                 ("k", C.c_void_p), ("v", C.c_void_p), ("ldkv", C.c_longlong),
                 ("kv_chunk_rows", C.c_longlong), ("Lk", C.c_int), ("pred_in_batch", C.c_int),
                 ("k0_pred", C.c_void_p), ("v0_pred", C.c_void_p), ("ld_pred", C.c_longlong),
-                ("Lk_pred", C.c_int), ("out", C.c_void_p), ("ldo", C.c_longlong)]
+                ("Lk_pred", C.c_int), ("out", C.c_void_p), ("ldo", C.c_longlong),
+                ("succ_in_batch", C.c_int)]
 
 
 class dp_ln_args(C.Structure):

@@ -204,6 +204,8 @@ static dp_status check_config(const dp_model_config* c) {
   if (c->text_len < 1 || c->text_in_dim < 1) return fail(DP_ERR_INVALID_ARG, "bad text shape");
   if (c->prec != DP_PREC_BF16 && c->prec != DP_PREC_FP32_VALIDATE)
     return fail(DP_ERR_INVALID_ARG, "bad precision");
+  if (c->neighbours != DP_NEIGHBOURS_PRED && c->neighbours != DP_NEIGHBOURS_BOTH)
+    return fail(DP_ERR_INVALID_ARG, "bad neighbours");
   if (c->prec == DP_PREC_BF16) {
     const int P = c->latent_ch * c->patch_t * c->patch_h * c->patch_w;
     if (hd != 64 && hd != 128) return fail(DP_ERR_INVALID_ARG, "bf16 path needs head_dim 64 or 128");
@@ -481,7 +483,8 @@ static dp_status run_step(dp_queue* q, const Plan& pl) {
       a.kv_chunk_rows = Lc;
       a.Lk = Lc;
       a.pred_in_batch = 1;
-      double keys = (double)n * Lc + (double)(n - 1) * Lc;
+      a.succ_in_batch = c.neighbours == DP_NEIGHBOURS_BOTH;
+      double keys = (double)n * Lc + (double)(n - 1) * Lc * (a.succ_in_batch ? 2 : 1);
       if (pl.head_pred == kPredCache) {
         a.k0_pred = static_cast<char*>(cache_rd) + (size_t)l * cache_layer * as;
         a.v0_pred = static_cast<char*>(cache_rd) + ((size_t)l * cache_layer + d) * as;

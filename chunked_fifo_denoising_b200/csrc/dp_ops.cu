@@ -70,8 +70,8 @@ dp_status dp_op_attention(const dp_attn_args* a, void* stream) {
   if (a->ldq < w || a->ldkv < w || a->ldo < w) return fail(DP_ERR_INVALID_ARG, "leading dimension too small");
   if (a->k0_pred && (!a->v0_pred || a->Lk_pred <= 0 || a->ld_pred < w))
     return fail(DP_ERR_INVALID_ARG, "bad predecessor buffer");
-  if (a->pred_in_batch && a->kv_chunk_rows <= 0)
-    return fail(DP_ERR_INVALID_ARG, "pred_in_batch needs per-chunk keys");
+  if ((a->pred_in_batch || a->succ_in_batch) && a->kv_chunk_rows <= 0)
+    return fail(DP_ERR_INVALID_ARG, "pred_in_batch / succ_in_batch need per-chunk keys");
   AttnParams p;
   memset(&p, 0, sizeof(p));
   p.f32 = a->dtype == DP_DT_F32;
@@ -93,6 +93,7 @@ dp_status dp_op_attention(const dp_attn_args* a, void* stream) {
   p.Lk_pred = a->k0_pred ? a->Lk_pred : 0;
   p.out = a->out;
   p.ldo = a->ldo;
+  p.succ_in_batch = a->succ_in_batch;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t err;
   if (a->dtype == DP_DT_F32) {

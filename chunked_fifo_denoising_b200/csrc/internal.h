@@ -49,6 +49,7 @@ struct AttnParams {
   int pred_in_batch;
   const void* k0_pred; const void* v0_pred; long long ld_pred; int Lk_pred;
   void* out; long long ldo;
+  int succ_in_batch;              // chunk c < n_chunks-1 also reads chunk c+1's own keys
 };
 
 struct LnParams {

@@ -1,6 +1,7 @@
-// SIMT flash attention (fp32 arithmetic) over up to two key buffers per chunk:
-// the predecessor's K/V (in-batch rows of chunk c-1, or the persisted K/V for
-// the first chunk) and the chunk's own K/V, one joint online softmax, no
+// SIMT flash attention (fp32 arithmetic) over up to three key buffers per
+// chunk: the predecessor's K/V (in-batch rows of chunk c-1, or the persisted
+// K/V for the first chunk), the chunk's own K/V and, optionally, the
+// successor's (in-batch rows of chunk c+1); one joint online softmax, no
 // concatenation.  One thread per query row; key tiles staged in shared memory.
 // Used by the fp32 validation mode.
 #include "common.cuh"
@@ -28,7 +29,7 @@ __global__ void __launch_bounds__(SA_Q) attn_simt_kernel(AttnParams p) {
   }
   float m = -INFINITY, l = 0.0f;
 
-  for (int src = 0; src < 2; ++src) {
+  for (int src = 0; src < 3; ++src) {  // predecessor, own, successor
     const T* Kb;
     const T* Vb;
     long long ld;
@@ -47,9 +48,15 @@ __global__ void __launch_bounds__(SA_Q) attn_simt_kernel(AttnParams p) {
       } else {
         continue;
       }
-    } else {
+    } else if (src == 1) {
       Kb = (const T*)p.k + (long long)c * p.kv_chunk_rows * p.ldkv;
       Vb = (const T*)p.v + (long long)c * p.kv_chunk_rows * p.ldkv;
+      ld = p.ldkv;
+      n = p.Lk;
+    } else {  // successor
+      if (!p.succ_in_batch || c + 1 >= p.n_chunks) continue;
+      Kb = (const T*)p.k + (long long)(c + 1) * p.kv_chunk_rows * p.ldkv;
+      Vb = (const T*)p.v + (long long)(c + 1) * p.kv_chunk_rows * p.ldkv;
       ld = p.ldkv;
       n = p.Lk;
     }

@@ -1,12 +1,14 @@
-// tcgen05 flash attention for sm_100a over up to two key buffers per chunk.
+// tcgen05 flash attention for sm_100a over up to three key buffers per chunk.
 //
 // DualParal write-up ("双重并行：让AI视频生成突破时长限制…", techwalker.com) §三:
 // a chunk's self-attention also reads the K/V of its neighbour, reused from a
 // cache rather than recomputed from a concatenated input.  Here the queries of
 // chunk c stream the key tiles of the predecessor buffer (chunk c-1's rows of
-// this batch, or the persisted K/V for the first chunk) and then of their own
-// buffer through one online softmax; the buffers are never concatenated.  The
-// same kernel with one shared buffer is the cross-attention to the prompt.
+// this batch, or the persisted K/V for the first chunk), then of their own
+// buffer and, with the bidirectional neighbourhood, of the successor (chunk
+// c+1's rows of this batch) through one online softmax; the buffers are never
+// concatenated.  The same kernel with one shared buffer is the cross-attention
+// to the prompt.
 //
 // CTA = 256 queries (two 128-row tiles A and B) of one (chunk, head), 10 warps:
 //   warp 0      TMA producer: Q_A, Q_B once; K and V tiles of 128 keys into two
@@ -55,8 +57,11 @@ struct AttnMaps {
   CUtensorMap q, k, v, kp, vp;
 };
 
-__device__ __forceinline__ int tile_valid(int j, int tiles_p, int n_p, int n_o) {
-  return j < tiles_p ? min(BKV, n_p - j * BKV) : min(BKV, n_o - (j - tiles_p) * BKV);
+// Key tiles of a chunk: predecessor [0, tp), own [tp, tp+to), successor after.
+__device__ __forceinline__ int tile_valid(int j, int tp, int n_p, int to, int n_o, int n_s) {
+  if (j < tp) return min(BKV, n_p - j * BKV);
+  if (j < tp + to) return min(BKV, n_o - (j - tp) * BKV);
+  return min(BKV, n_s - (j - tp - to) * BKV);
 }
 
 // Warp-uniform bounded wait: TMEM loads and stores that follow are
@@ -130,8 +135,10 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
     pred_cache = true;
   }
   const int n_o = p.Lk;
+  const int n_s = (p.succ_in_batch && c + 1 < p.n_chunks) ? p.Lk : 0;
   const int tiles_p = (n_p + BKV - 1) / BKV;
-  const int nt = tiles_p + (n_o + BKV - 1) / BKV;
+  const int tiles_o = (n_o + BKV - 1) / BKV;
+  const int nt = tiles_p + tiles_o + (n_s + BKV - 1) / BKV;
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
@@ -184,10 +191,14 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
             mv = &maps.v;
             row = (int)((c - 1) * p.kv_chunk_rows) + j * BKV;
           }
-        } else {
+        } else if (j < tiles_p + tiles_o) {
           mk = &maps.k;
           mv = &maps.v;
           row = (int)(c * p.kv_chunk_rows) + (j - tiles_p) * BKV;
+        } else {  // successor: chunk c+1's own rows of this batch
+          mk = &maps.k;
+          mv = &maps.v;
+          row = (int)((c + 1) * p.kv_chunk_rows) + (j - tiles_p - tiles_o) * BKV;
         }
         if (use > 0 && !mbar_wait(&k_empty[st], (use - 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
         mbar_arrive_expect_tx(&k_full[st], C::T_BYTES);
@@ -288,7 +299,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
 #pragma unroll
         for (int i = 0; i < 4; ++i) tmem_ld32_nowait(tS + i * 32, *reinterpret_cast<float(*)[32]>(s + i * 32));
         tmem_wait_ld();
-        const int valid = tile_valid(j, tiles_p, n_p, n_o);
+        const int valid = tile_valid(j, tiles_p, n_p, tiles_o, n_o, n_s);
         if (valid < BKV) {
 #pragma unroll
           for (int i = 0; i < 128; ++i)

@@ -51,13 +51,14 @@ class Model:
     text_len, text_in_dim, latent_ch, patch_t, patch_h, patch_w.
     """
 
-    def __init__(self, shape, precision="bf16", stream=None):
+    def __init__(self, shape, precision="bf16", stream=None, neighbours="pred"):
         self.shape = shape
         self.cfg = B.dp_model_config(
             shape.n_layers, shape.dim, shape.n_heads, shape.ffn_dim, shape.freq_dim,
             shape.latent_ch, shape.patch_t, shape.patch_h, shape.patch_w, shape.text_len,
             shape.text_in_dim,
-            B.DP_PREC_BF16 if precision == "bf16" else B.DP_PREC_FP32_VALIDATE)
+            B.DP_PREC_BF16 if precision == "bf16" else B.DP_PREC_FP32_VALIDATE,
+            B.DP_NEIGHBOURS_BOTH if neighbours == "both" else B.DP_NEIGHBOURS_PRED)
         self.handle = C.c_void_p()
         B.check(B.dp_model_create(self.cfg, _stream_handle(stream), self.handle), "dp_model_create")
         self.queues = []

@@ -76,6 +76,15 @@ typedef enum {
   DP_LOC_HOST = 1
 } dp_loc;
 
+/* Which neighbours a chunk's self-attention reads besides its own tokens.
+ * PRED: the preceding chunk k-1 (its K/V from this pass, or persisted from the
+ * previous step once it has left the queue).  BOTH: also the following chunk
+ * k+1 when it is queued in the same pass (the chunk pushed last has none). */
+typedef enum {
+  DP_NEIGHBOURS_PRED = 0,
+  DP_NEIGHBOURS_BOTH = 1
+} dp_neighbours;
+
 /* Model shape.  dim % n_heads == 0; head_dim = dim / n_heads must be 16, 32,
  * 64 or 128 (the production path needs 64 or 128); freq_dim even;
  * patch = patch_t x patch_h x patch_w over latent_ch channels. */
@@ -90,6 +99,7 @@ typedef struct {
   int text_len;     /* prompt tokens                                  */
   int text_in_dim;  /* prompt feature width; != dim adds a projection */
   dp_precision prec;
+  dp_neighbours neighbours;
 } dp_model_config;
 
 /* Queue shape.  One chunk = latent_ch x frames_per_chunk x lat_h x lat_w fp32,

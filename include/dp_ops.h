@@ -71,7 +71,8 @@ DP_API dp_status dp_op_gemm(const dp_gemm_args* a, void* stream);
  *   - if pred_in_batch and c > 0: the own keys of chunk c - 1 (the
  *     neighbour's K/V already computed in this batch), read in place;
  *   - for c = 0: the Lk_pred keys k0_pred/v0_pred when not NULL (the
- *     neighbour's persisted K/V from the previous step).
+ *     neighbour's persisted K/V from the previous step);
+ *   - if succ_in_batch and c < n_chunks - 1: the own keys of chunk c + 1.
  * Queries of chunk c are rows [c * Lq, (c + 1) * Lq) of q.  Head h uses
  * columns [h * head_dim, (h + 1) * head_dim) of q, k, v and out.
  * bf16 requires head_dim 64 or 128 (tcgen05 path); f32 requires head_dim <= 128. */
@@ -83,6 +84,7 @@ typedef struct {
   int pred_in_batch;
   const void* k0_pred; const void* v0_pred; long long ld_pred; int Lk_pred;
   void* out; long long ldo;
+  int succ_in_batch;
 } dp_attn_args;
 DP_API dp_status dp_op_attention(const dp_attn_args* a, void* stream);
 

@@ -164,6 +164,28 @@ def attention(q, k, v, n_heads):
     return out
 
 
+def self_attention_with_neighbours(q, k, v, k_pred, v_pred, k_succ, v_succ, n_heads):
+    """Self-attention of a chunk over its predecessor's, its own and its
+    successor's K/V in one joint softmax (the key set written out as the
+    concatenation).  Either neighbour may be None.
+
+    DualParal write-up §三: processing chunk B_i with both neighbours,
+    [B_{i-1}, B_i, B_{i+1}], is the starting point; the neighbours enter only
+    through self-attention.  This is the bidirectional reading of the
+    neighbourhood (the predecessor-only reading is the default).
+    """
+    ks, vs = [], []
+    if k_pred is not None:
+        ks.append(k_pred)
+        vs.append(v_pred)
+    ks.append(k)
+    vs.append(v)
+    if k_succ is not None:
+        ks.append(k_succ)
+        vs.append(v_succ)
+    return attention(q, np.concatenate(ks), np.concatenate(vs), n_heads)
+
+
 def self_attention_with_predecessor(q, k, v, k_pred, v_pred, n_heads):
     """A chunk's self-attention: its queries see its own keys plus the K/V of
     the chunk before it, in one joint softmax.
@@ -204,7 +226,7 @@ def text_kv(text, p, n_layers):
 # ---------------------------------------------------------------------------
 
 def velocity(latents, levels, chunk_ids, pred_kv, p, tkv, shape, T, use_pred=True,
-             keep_kv_of=None):
+             keep_kv_of=None, neighbours="pred"):
     """Model output v for every queued chunk of one step.
 
     latents   list of [C][F][H][W] arrays, one per queued chunk, ordered by
@@ -214,8 +236,11 @@ def velocity(latents, levels, chunk_ids, pred_kv, p, tkv, shape, T, use_pred=Tru
               self-attention K/V of the chunk just before the first queued one.
     tkv       ``text_kv`` output.
     shape     synth.ModelShape.
-    use_pred  False disables the predecessor link entirely.
+    use_pred  False disables the neighbour links entirely.
     keep_kv_of  index into the batch whose per-layer (K, V) are returned.
+    neighbours  "pred" (the predecessor only) or "both" (also the successor
+              k+1, read from this pass when it is queued; the chunk pushed last
+              has none).
 
     Returns (v list, kept kv list-or-None).
 
@@ -263,7 +288,10 @@ def velocity(latents, levels, chunk_ids, pred_kv, p, tkv, shape, T, use_pred=Tru
                 kp, vp = (np.asarray(a, np.float64) for a in pred_kv[l])
             else:
                 kp = vp = None
-            o = self_attention_with_predecessor(q[i], k[i], v[i], kp, vp, H)
+            ksu = vsu = None
+            if use_pred and neighbours == "both" and i + 1 < n:
+                ksu, vsu = k[i + 1], v[i + 1]
+            o = self_attention_with_neighbours(q[i], k[i], v[i], kp, vp, ksu, vsu, H)
             x[i] = x[i] + g_a * linear(o, p["layer.o.w"][l], p["layer.o.b"][l])
             # cross-attention to the prompt (no modulation, no gate)
             h = layer_norm(x[i])
@@ -283,11 +311,11 @@ def velocity(latents, levels, chunk_ids, pred_kv, p, tkv, shape, T, use_pred=Tru
     return vs, kept
 
 
-def make_velocity_fn(p, text, shape, T, use_pred=True):
+def make_velocity_fn(p, text, shape, T, use_pred=True, neighbours="pred"):
     """Binds parameters and the prompt into the callable the queue expects."""
     tkv = text_kv(text, p, shape.n_layers)
 
     def fn(latents, levels, chunk_ids, pred_kv, keep_kv_of):
         return velocity(latents, levels, chunk_ids, pred_kv, p, tkv, shape, T,
-                        use_pred=use_pred, keep_kv_of=keep_kv_of)
+                        use_pred=use_pred, keep_kv_of=keep_kv_of, neighbours=neighbours)
     return fn

@@ -162,7 +162,7 @@ def test_gemm_full_size_sampled_rows(name, M, N, K):
 # ---------------------------------------------------------------------------
 
 def run_attn(q, k, v, n_chunks, Lq, H, hd, Lk, kv_chunk_rows, pred_in_batch, kp=None, vp=None,
-             dtype=None):
+             dtype=None, succ=0):
     out = torch.empty((n_chunks * Lq, H * hd), device="cuda", dtype=q.dtype)
     a = B.dp_attn_args()
     a.dtype = B.DP_DT_BF16 if q.dtype == torch.bfloat16 else B.DP_DT_F32
@@ -173,14 +173,16 @@ def run_attn(q, k, v, n_chunks, Lq, H, hd, Lk, kv_chunk_rows, pred_in_batch, kp=
     if kp is not None:
         a.k0_pred, a.v0_pred, a.ld_pred, a.Lk_pred = kp.data_ptr(), vp.data_ptr(), kp.stride(0), kp.shape[0]
     a.out, a.ldo = out.data_ptr(), out.stride(0)
+    a.succ_in_batch = succ
     st = B.dp_op_attention(a, torch.cuda.current_stream().cuda_stream)
     assert st == 0, B.dp_last_error()
     assert B.dp_op_check(torch.cuda.current_stream().cuda_stream) == 0, B.dp_last_error()
     return out
 
 
-def oracle_self_attention(q, k, v, n, Lc, H, kp, vp, rows=None):
-    """Per chunk: own keys plus the predecessor's (in batch, or kp/vp for chunk 0)."""
+def oracle_self_attention(q, k, v, n, Lc, H, kp, vp, rows=None, succ=False):
+    """Per chunk: own keys plus the predecessor's (in batch, or kp/vp for chunk 0)
+    and, with succ, the successor's (in batch)."""
     outs = []
     for c in range(n):
         sl = slice(c * Lc, (c + 1) * Lc)
@@ -189,14 +191,18 @@ def oracle_self_attention(q, k, v, n, Lc, H, kp, vp, rows=None):
             pk, pv = k[(c - 1) * Lc:c * Lc], v[(c - 1) * Lc:c * Lc]
         else:
             pk, pv = kp, vp
-        outs.append(dit.self_attention_with_predecessor(qq, k[sl], v[sl], pk, pv, H))
+        sk = sv = None
+        if succ and c + 1 < n:
+            sk, sv = k[(c + 1) * Lc:(c + 2) * Lc], v[(c + 1) * Lc:(c + 2) * Lc]
+        outs.append(dit.self_attention_with_neighbours(qq, k[sl], v[sl], pk, pv, sk, sv, H))
     return np.concatenate(outs)
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("hd,Lc,n,cached", [(64, 200, 3, True), (128, 333, 2, False),
-                                            (128, 130, 4, True)])
-def test_self_attention_two_buffers(dtype, hd, Lc, n, cached):
+@pytest.mark.parametrize("hd,Lc,n,cached,succ", [(64, 200, 3, True, False), (128, 333, 2, False, False),
+                                                 (128, 130, 4, True, False), (128, 200, 3, True, True),
+                                                 (64, 333, 2, False, True)])
+def test_self_attention_neighbour_buffers(dtype, hd, Lc, n, cached, succ):
     H = 2
     d = H * hd
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
@@ -205,9 +211,10 @@ def test_self_attention_two_buffers(dtype, hd, Lc, n, cached):
     cache = gen((Lc, 2 * d), 1.0, tdt, seed=31) if cached else None
     kp = cache[:, :d] if cached else None
     vp = cache[:, d:] if cached else None
-    out = run_attn(q, k, v, n, Lc, H, hd, Lc, Lc, 1, kp, vp)
+    out = run_attn(q, k, v, n, Lc, H, hd, Lc, Lc, 1, kp, vp, succ=int(succ))
     ref = oracle_self_attention(f64(q), f64(k), f64(v), n, Lc, H,
-                                None if kp is None else f64(kp), None if vp is None else f64(vp))
+                                None if kp is None else f64(kp), None if vp is None else f64(vp),
+                                succ=succ)
     assert rel_l2(f64(out), ref) < (1e-2 if dtype == "bf16" else 1e-5)
 
 
@@ -223,15 +230,17 @@ def test_cross_attention_shared_keys(dtype):
     assert rel_l2(f64(out), ref) < (1e-2 if dtype == "bf16" else 1e-5)
 
 
-def test_self_attention_full_size_sampled_rows():
+@pytest.mark.parametrize("succ", [False, True])
+def test_self_attention_full_size_sampled_rows(succ):
     """Wan-1.3B steady state: 50 chunks of 3120 tokens, 12 heads of 128, every
-    chunk with its predecessor (chunk 0 from the persisted cache)."""
+    chunk with its predecessor (chunk 0 from the persisted cache), and with the
+    bidirectional neighbourhood also its successor."""
     n, Lc, H, hd = 50, 3120, 12, 128
     d = H * hd
     qkv = gen((n * Lc, 3 * d), 1.0, torch.bfloat16, seed=40)
     q, k, v = qkv[:, :d], qkv[:, d:2 * d], qkv[:, 2 * d:]
     cache = gen((Lc, 2 * d), 1.0, torch.bfloat16, seed=41)
-    out = run_attn(q, k, v, n, Lc, H, hd, Lc, Lc, 1, cache[:, :d], cache[:, d:])
+    out = run_attn(q, k, v, n, Lc, H, hd, Lc, Lc, 1, cache[:, :d], cache[:, d:], succ=int(succ))
     rows = np.array([0, 1, 127, 128, 1000, 3119])
     qf, kf, vf = f64(q), f64(k), f64(v)
     for c in (0, 1, 17, 49):
@@ -240,7 +249,10 @@ def test_self_attention_full_size_sampled_rows():
             pk, pv = kf[(c - 1) * Lc:c * Lc], vf[(c - 1) * Lc:c * Lc]
         else:
             pk, pv = f64(cache[:, :d]), f64(cache[:, d:])
-        ref = dit.self_attention_with_predecessor(qf[sl][rows], kf[sl], vf[sl], pk, pv, H)
+        sk = sv = None
+        if succ and c + 1 < n:
+            sk, sv = kf[(c + 1) * Lc:(c + 2) * Lc], vf[(c + 1) * Lc:(c + 2) * Lc]
+        ref = dit.self_attention_with_neighbours(qf[sl][rows], kf[sl], vf[sl], pk, pv, sk, sv, H)
         assert rel_l2(f64(out[sl][rows]), ref) < 1e-2, c
 
 

@@ -39,24 +39,25 @@ def bf16_round(x):
     return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16).float().numpy()
 
 
-def make(w, precision, params=None, text=None, n_chunks=None, T=None, ready=2):
+def make(w, precision, params=None, text=None, n_chunks=None, T=None, ready=2, neighbours="pred"):
     from chunked_fifo_denoising_b200 import Model, Queue
     m, q = w.model, w.queue
     params = synth.make_params(m) if params is None else params
     text = synth.make_text(m) if text is None else text
-    model = Model(m, precision)
+    model = Model(m, precision, neighbours=neighbours)
     model.set_params(params)
     queue = Queue(model, text, q.T if T is None else T, q.frames_per_chunk, q.lat_h, q.lat_w,
                   q.n_chunks if n_chunks is None else n_chunks, ready_capacity=ready)
     return model, queue, params, text
 
 
-def test_tiny_fp32_stream_matches_oracle():
+@pytest.mark.parametrize("neighbours", ["pred", "both"])
+def test_tiny_fp32_stream_matches_oracle(neighbours):
     w = synth.WORKLOADS["tiny_fp32"]
     m, q = w.model, w.queue
-    model, queue, p, text = make(w, "fp32")
+    model, queue, p, text = make(w, "fp32", neighbours=neighbours)
     noise = [synth.make_noise(m, q, k) for k in range(q.n_chunks)]
-    fn = dit.make_velocity_fn(p, text, m, q.T)
+    fn = dit.make_velocity_fn(p, text, m, q.T, neighbours=neighbours)
     ready, traces = fifo.run_stream(fn, lambda k: noise[k], q.T, q.n_chunks)
     out = np.empty(q.chunk_shape(m), np.float32)
     got = {}
@@ -113,7 +114,7 @@ def test_bookkeeping_exact_on_every_schedule(name):
     model.close()
 
 
-def _one_step_parity(w, n_layers=None, n_occ=3, seed_state=7):
+def _one_step_parity(w, n_layers=None, n_occ=3, seed_state=7, neighbours="pred"):
     """Queue state just before a step: chunks at levels 1 .. n_occ (no push),
     the head's predecessor K/V persisted; compare one GPU step with the oracle."""
     if n_layers is not None:
@@ -123,7 +124,7 @@ def _one_step_parity(w, n_layers=None, n_occ=3, seed_state=7):
     n_chunks = 20
     head = n_chunks - n_occ
     step = head + T - 1              # the head chunk is at level 1
-    model, queue, p, text = make(w, "bf16", n_chunks=n_chunks)
+    model, queue, p, text = make(w, "bf16", n_chunks=n_chunks, neighbours=neighbours)
     rng = np.random.default_rng(seed_state)
     lat = rng.standard_normal((n_occ,) + q.chunk_shape(m)).astype(np.float32)
     Lc = q.tokens_per_chunk(m)
@@ -140,7 +141,7 @@ def _one_step_parity(w, n_layers=None, n_occ=3, seed_state=7):
     new_kv, kv_id = queue.read_pred_kv()
     assert kv_id == head
     # oracle
-    fn = dit.make_velocity_fn(p, text, m, T)
+    fn = dit.make_velocity_fn(p, text, m, T, neighbours=neighbours)
     st = fifo.QueueState(T=T, n_chunks=n_chunks, step=step, next_id=n_chunks,
                          entries=[fifo.Entry(head + i, 1 + i, lat[i].astype(np.float64)) for i in range(n_occ)],
                          pred_id=head - 1, pred_kv=[(kv[l, 0], kv[l, 1]) for l in range(m.n_layers)])
@@ -163,6 +164,11 @@ def _one_step_parity(w, n_layers=None, n_occ=3, seed_state=7):
 
 def test_bf16_step_small():
     _one_step_parity(synth.WORKLOADS["small_bf16"])
+
+
+def test_bf16_step_small_bidirectional():
+    """The bidirectional neighbourhood: chunk k also reads chunk k+1's K/V."""
+    _one_step_parity(synth.WORKLOADS["small_bf16"], neighbours="both")
 
 
 def test_bf16_step_wan13b_shapes_two_layers():

@@ -410,3 +410,41 @@ def test_level_changes_velocity(tiny):
     (va,), _ = fn([x], [1], [0], None, None)
     (vb,), _ = fn([x], [4], [0], None, None)
     assert not np.allclose(va, vb)
+
+
+def test_three_buffer_attention_equals_streaming_and_concat():
+    """Bidirectional neighbourhood: [pred; own; succ] from three buffers equals
+    one streamed softmax over them and brute force over the concatenation; the
+    order of the buffers is irrelevant."""
+    rng = np.random.default_rng(9)
+    q, k, v = rng.normal(size=(4, 8)), rng.normal(size=(5, 8)), rng.normal(size=(5, 8))
+    kp, vp = rng.normal(size=(5, 8)), rng.normal(size=(5, 8))
+    ks, vs = rng.normal(size=(5, 8)), rng.normal(size=(5, 8))
+    got = dit.self_attention_with_neighbours(q, k, v, kp, vp, ks, vs, 2)
+    assert np.allclose(got, streaming_two_buffer(q, [(ks, vs), (kp, vp), (k, v)], 2), rtol=1e-6, atol=1e-12)
+    assert np.allclose(got, brute_attention(q, np.vstack([kp, k, ks]), np.vstack([vp, v, vs]), 2), atol=1e-12)
+    # no successor: the predecessor-only form
+    assert np.allclose(dit.self_attention_with_neighbours(q, k, v, kp, vp, None, None, 2),
+                       dit.self_attention_with_predecessor(q, k, v, kp, vp, 2), atol=1e-15)
+
+
+def test_bidirectional_link_reaches_both_ways(tiny):
+    """With both neighbours, changing chunk 2 changes chunks 0..4 (one hop per
+    layer each way, 2 layers) and leaves chunk 5 unchanged."""
+    p, text, noise = tiny
+    L = W.model.n_layers
+    fn = dit.make_velocity_fn(p, text, W.model, T=8, neighbours="both")
+    lat = [np.asarray(noise[k % 6], np.float64) for k in range(6)]
+    lv, ids = [1, 2, 3, 4, 5, 6], list(range(6))
+    v0, _ = fn(lat, lv, ids, None, None)
+    lat2 = list(lat)
+    lat2[2] = lat[2] + 0.5
+    v1, _ = fn(lat2, lv, ids, None, None)
+    for k in range(2 - L, 2 + L + 1):
+        assert not np.allclose(v0[k], v1[k]), k
+    assert np.array_equal(v0[5], v1[5])
+    # the predecessor-only model never looks forward
+    fp = dit.make_velocity_fn(p, text, W.model, T=8)
+    w0, _ = fp(lat, lv, ids, None, None)
+    w1, _ = fp(lat2, lv, ids, None, None)
+    assert np.array_equal(w0[0], w1[0]) and np.array_equal(w0[1], w1[1])
