@@ -247,6 +247,9 @@ def run_ours(args, w):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local))
+    if args.qk_norm_rope:
+        import synth as _s
+        w = _s.with_qk_norm_rope(w)
     m, q = w.model, w.queue
     T = q.T
     occ = T
@@ -258,6 +261,8 @@ def run_ours(args, w):
     for name, shape, per_layer in synth.param_specs(m):
         for l in range(m.n_layers if per_layer else 1):
             t = torch.randn(shape, generator=g, device="cuda") * 0.02
+            if name.endswith("norm.w"):
+                t += 1.0
             model.set_param(name, t, l)
             del t
     text = torch.randn((m.text_len, m.text_in_dim), generator=g, device="cuda")
@@ -338,6 +343,7 @@ def run_ours(args, w):
                        "tokens_per_step": occ * q.tokens_per_chunk(m), "frames_per_step": frames,
                        "layers": m.n_layers, "dim": m.dim, "ffn": m.ffn_dim, "heads": m.n_heads,
                        "text_tokens": m.text_len, "neighbours": args.neighbours,
+                       "qk_norm_rope": bool(args.qk_norm_rope),
                        "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (fp32 residual stream alone is "
                              f"{occ * q.tokens_per_chunk(m) * m.dim * 4 / 1e6:.0f} MB)"},
@@ -375,6 +381,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="wan1.3b_480p")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--qk-norm-rope", action="store_true",
+                    help="per-head QK RMSNorm and 3-D rotary positions in self-attention")
     ap.add_argument("--neighbours", default="pred", choices=["pred", "both"],
                     help="self-attention neighbourhood: predecessor only, or also the successor")
     args = ap.parse_args()

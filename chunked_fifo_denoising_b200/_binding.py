@@ -33,8 +33,9 @@ PARAM_IDS = {
     "layer.cq.w": 19, "layer.cq.b": 20, "layer.ck.w": 21, "layer.ck.b": 22,
     "layer.cv.w": 23, "layer.cv.b": 24, "layer.co.w": 25, "layer.co.b": 26,
     "layer.ffn1.w": 27, "layer.ffn1.b": 28, "layer.ffn2.w": 29, "layer.ffn2.b": 30,
+    "layer.qnorm.w": 31, "layer.knorm.w": 32,
 }
-DP_PARAM_COUNT = 31
+DP_PARAM_COUNT = 33
 
 
 class dp_model_config(C.Structure):
@@ -42,7 +43,7 @@ class dp_model_config(C.Structure):
                 ("ffn_dim", C.c_int), ("freq_dim", C.c_int), ("latent_ch", C.c_int),
                 ("patch_t", C.c_int), ("patch_h", C.c_int), ("patch_w", C.c_int),
                 ("text_len", C.c_int), ("text_in_dim", C.c_int), ("prec", C.c_int),
-                ("neighbours", C.c_int)]
+                ("neighbours", C.c_int), ("qk_norm_rope", C.c_int)]
 
 
 class dp_queue_config(C.Structure):

@@ -177,6 +177,7 @@ static long long param_numel(const dp_model_config& c, dp_param id) {
     case DP_L_FFN1_B: return F;
     case DP_L_FFN2_W: return d * F;
     case DP_L_FFN2_B: return d;
+    case DP_L_QNORM_W: case DP_L_KNORM_W: return c.qk_norm_rope ? d : 0;
     default: return -1;
   }
 }
@@ -206,6 +207,8 @@ static dp_status check_config(const dp_model_config* c) {
     return fail(DP_ERR_INVALID_ARG, "bad precision");
   if (c->neighbours != DP_NEIGHBOURS_PRED && c->neighbours != DP_NEIGHBOURS_BOTH)
     return fail(DP_ERR_INVALID_ARG, "bad neighbours");
+  if (c->qk_norm_rope != 0 && c->qk_norm_rope != 1) return fail(DP_ERR_INVALID_ARG, "bad qk_norm_rope");
+  if (c->qk_norm_rope && hd < 6) return fail(DP_ERR_INVALID_ARG, "rotary positions need head_dim >= 6");
   if (c->prec == DP_PREC_BF16) {
     const int P = c->latent_ch * c->patch_t * c->patch_h * c->patch_w;
     if (hd != 64 && hd != 128) return fail(DP_ERR_INVALID_ARG, "bf16 path needs head_dim 64 or 128");
@@ -434,6 +437,7 @@ static dp_status run_step(dp_queue* q, const Plan& pl) {
   void* cache_wr = q->cache[1 - q->cache_cur].p;
   const long long cache_layer = (long long)Lc * 2 * d;  // elements per layer
   char* qkv = q->qkv.as<char>();
+  const bool rope_fused = c.qk_norm_rope && !f32 && d % 256 == 0 && (m->hd == 64 || m->hd == 128);
   for (int l = 0; l < L; ++l) {
     float* mt = modtab + (long long)l * 6 * d;
     // --- self-attention block -------------------------------------------
@@ -465,7 +469,53 @@ static dp_status run_step(dp_queue* q, const Plan& pl) {
         e.cache_col0 = d;
         e.ldc = 2 * d;
       }
+      // fused into the tensor-core epilogue when every 128-column half of a
+      // 256-column tile holds whole heads of one part (q or k): d % 256 == 0
+      if (rope_fused) {
+        e.rope = 1;
+        e.rows_per_chunk = Lc;
+        e.rope_d = d;
+        e.rope_hd = m->hd;
+        e.rope_Fq = q->rope_Fq;
+        e.rope_Hq = qc.lat_h / c.patch_h;
+        e.rope_Wq = qc.lat_w / c.patch_w;
+        e.rope_nt = q->rope_nt;
+        e.rope_nh = q->rope_nh;
+        e.q_w = m->wf(DP_L_QNORM_W, l);
+        e.k_w = m->wf(DP_L_KNORM_W, l);
+        e.rope_t = q->rope_t.as<float2>();
+        e.rope_y = q->rope_y.as<float2>();
+        e.rope_x = q->rope_x.as<float2>();
+      }
       DP_TRY(st.gemm(q->h.p, d, m->w(DP_L_QKV_W, l), M, 3 * d, d, e));
+    }
+    if (c.qk_norm_rope && !rope_fused) {  // separate in-place kernel (fp32 mode, other widths)
+      RopeParams rp;
+      memset(&rp, 0, sizeof(rp));
+      rp.f32 = f32;
+      rp.qkv = qkv;
+      rp.ld = 3 * d;
+      rp.M = M;
+      rp.d = d;
+      rp.n_heads = m->H;
+      rp.Lc = Lc;
+      rp.Fq = q->rope_Fq;
+      rp.Hq = qc.lat_h / c.patch_h;
+      rp.Wq = qc.lat_w / c.patch_w;
+      rp.nt = q->rope_nt;
+      rp.nh = q->rope_nh;
+      rp.q_w = m->wf(DP_L_QNORM_W, l);
+      rp.k_w = m->wf(DP_L_KNORM_W, l);
+      rp.rope_t = q->rope_t.as<float2>();
+      rp.rope_y = q->rope_y.as<float2>();
+      rp.rope_x = q->rope_x.as<float2>();
+      if (pl.writes_cache) {  // the persisted K of the head chunk holds the rotated keys
+        rp.cache = static_cast<char*>(cache_wr) + (size_t)l * cache_layer * as;
+        rp.ldc = 2 * d;
+      }
+      DP_TRY(q->timer.begin(KC_OTHER));
+      DP_CK(qk_norm_rope(rp, s));
+      DP_TRY(q->timer.end(0.0, (double)M * 2 * d * 2 * as));
     }
     {
       AttnParams a;
@@ -615,6 +665,22 @@ static dp_status upload_tables(dp_queue* q, const Plan& pl) {
     q->h_dsig[i] = (float)((double)(j - 1) / T - (double)j / T);
   }
   cudaStream_t s = q->m->stream;
+  if (q->m->cfg.qk_norm_rope) {
+    // temporal rotary table of this step: absolute frame (chunk id * Fq + f)
+    const int nt = q->rope_nt, Fq = q->rope_Fq;
+    for (int c = 0; c < pl.n; ++c)
+      for (int f = 0; f < Fq; ++f) {
+        const double pos = (double)(pl.head + c) * Fq + f;
+        for (int l = 0; l < nt; ++l) {
+          const double a = std::fmod(pos * std::pow(10000.0, -(double)l / nt), 2.0 * M_PI);
+          float* e = q->h_rope_t + 2 * (((size_t)c * Fq + f) * nt + l);
+          e[0] = (float)std::cos(a);
+          e[1] = (float)std::sin(a);
+        }
+      }
+    DP_CK(cudaMemcpyAsync(q->rope_t.p, q->h_rope_t, (size_t)pl.n * Fq * nt * 2 * sizeof(float),
+                          cudaMemcpyHostToDevice, s));
+  }
   DP_CK(cudaMemcpyAsync(q->d_sel.p, q->h_sel, pl.n * sizeof(int), cudaMemcpyHostToDevice, s));
   DP_CK(cudaMemcpyAsync(q->d_slot.p, q->h_slot, pl.n * sizeof(int), cudaMemcpyHostToDevice, s));
   DP_CK(cudaMemcpyAsync(q->d_dsig.p, q->h_dsig, pl.n * sizeof(float), cudaMemcpyHostToDevice, s));
@@ -624,8 +690,10 @@ static dp_status upload_tables(dp_queue* q, const Plan& pl) {
 
 static void free_queue(dp_queue* q) {
   DevBuf* bufs[] = {&q->ring, &q->x, &q->h, &q->qkv, &q->attn, &q->u, &q->textkv, &q->cache[0],
-                    &q->cache[1], &q->modtab, &q->hmod, &q->d_sel, &q->d_slot, &q->d_dsig};
+                    &q->cache[1], &q->modtab, &q->hmod, &q->d_sel, &q->d_slot, &q->d_dsig,
+                    &q->rope_t, &q->rope_y, &q->rope_x};
   for (DevBuf* b : bufs) dev_free(*b);
+  if (q->h_rope_t) cudaFreeHost(q->h_rope_t);
   if (q->h_sel) cudaFreeHost(q->h_sel);
   if (q->h_slot) cudaFreeHost(q->h_slot);
   if (q->h_dsig) cudaFreeHost(q->h_dsig);
@@ -755,16 +823,43 @@ dp_status dp_queue_init(dp_model* m, const dp_queue_config* qc, const float* tex
   QA(q->d_sel, (size_t)qc->T * 4, "chunk levels");
   QA(q->d_slot, (size_t)qc->T * 4, "chunk slots");
   QA(q->d_dsig, (size_t)qc->T * 4, "chunk sigma steps");
+  if (c.qk_norm_rope) {
+    q->rope_Fq = qc->frames_per_chunk / c.patch_t;
+    q->rope_nh = (m->hd / 2) / 3;
+    q->rope_nt = m->hd / 2 - 2 * q->rope_nh;
+    QA(q->rope_t, (size_t)qc->T * q->rope_Fq * q->rope_nt * 2 * 4, "temporal rotary table");
+    QA(q->rope_y, (size_t)(qc->lat_h / c.patch_h) * q->rope_nh * 2 * 4, "row rotary table");
+    QA(q->rope_x, (size_t)(qc->lat_w / c.patch_w) * q->rope_nh * 2 * 4, "column rotary table");
+  }
 #undef QA
   if (s == DP_OK) {
     cudaError_t e = cudaMallocHost(&q->h_sel, qc->T * sizeof(int));
     if (e == cudaSuccess) e = cudaMallocHost(&q->h_slot, qc->T * sizeof(int));
     if (e == cudaSuccess) e = cudaMallocHost(&q->h_dsig, qc->T * sizeof(float));
+    if (e == cudaSuccess && c.qk_norm_rope)
+      e = cudaMallocHost(&q->h_rope_t, (size_t)qc->T * q->rope_Fq * q->rope_nt * 2 * sizeof(float));
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&q->table_ev, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventRecord(q->table_ev, m->stream);
     if (e != cudaSuccess) s = fail(DP_ERR_OOM, "pinned staging: %s", cudaGetErrorString(e));
   }
   if (s == DP_OK) s = build_tables(q, text, text_loc);
+  if (s == DP_OK && c.qk_norm_rope) {
+    // row and column rotary tables, fixed for the queue: angle = pos * 10000^(-l/nh)
+    const int nh = q->rope_nh;
+    for (int axis = 0; axis < 2 && s == DP_OK; ++axis) {
+      const int npos = axis == 0 ? qc->lat_h / c.patch_h : qc->lat_w / c.patch_w;
+      std::vector<float> tab((size_t)npos * nh * 2);
+      for (int pos = 0; pos < npos; ++pos)
+        for (int l = 0; l < nh; ++l) {
+          const double a = pos * std::pow(10000.0, -(double)l / nh);
+          tab[2 * ((size_t)pos * nh + l)] = (float)std::cos(a);
+          tab[2 * ((size_t)pos * nh + l) + 1] = (float)std::sin(a);
+        }
+      cudaError_t e = cudaMemcpy(axis == 0 ? q->rope_y.p : q->rope_x.p, tab.data(),
+                                 tab.size() * sizeof(float), cudaMemcpyHostToDevice);
+      if (e != cudaSuccess) s = fail(DP_ERR_CUDA, "rotary tables: %s", cudaGetErrorString(e));
+    }
+  }
   if (s != DP_OK) {
     std::string msg = dp_last_error();
     free_queue(q);

@@ -39,6 +39,12 @@ struct EpiParams {
   const int* chunk_slot;          // [batch chunk] -> ring slot
   const float* dsig;              // [batch chunk] -> sigma_{j-1} - sigma_j
   int lat_c, lat_f, lat_h, lat_w, pt, ph, pw;
+  // QKV epilogue with per-head RMSNorm + rotary positions on the q and k
+  // column blocks [0, 2 * rope_d) (bf16 tensor-core path; rows_per_chunk = Lc)
+  int rope;
+  int rope_d, rope_hd, rope_Fq, rope_Hq, rope_Wq, rope_nt, rope_nh;
+  const float* q_w; const float* k_w;
+  const float2* rope_t; const float2* rope_y; const float2* rope_x;
 };
 
 struct AttnParams {
@@ -75,6 +81,21 @@ cudaError_t attention_tc(const AttnParams& p, int* status, cudaStream_t s);
 bool attention_tc_supported(const AttnParams& p);
 
 cudaError_t layernorm_mod(const LnParams& p, cudaStream_t s);
+
+// Per-head RMSNorm + 3-D rotary positions applied in place to the q and k
+// column blocks of a [M][ld] qkv buffer (q at col 0, k at col d).  Tables hold
+// (cos, sin) float pairs: rope_t [n_chunks * Fq][nt], rope_y [Hq][nh],
+// rope_x [Wq][nw].  Rows of batch chunk 0 with cache != null also write the
+// result of k to cache[row * ldc + col].
+struct RopeParams {
+  int f32;
+  void* qkv; long long ld;
+  int M, d, n_heads, Lc, Fq, Hq, Wq, nt, nh;
+  const float* q_w; const float* k_w;
+  const float2* rope_t; const float2* rope_y; const float2* rope_x;
+  void* cache; long long ldc;
+};
+cudaError_t qk_norm_rope(const RopeParams& p, cudaStream_t s);
 
 // ring [slots][C][F][H][W] fp32 -> patches [M][P] (float or bf16)
 cudaError_t gather_patches(const float* ring, long long chunk_numel, const int* chunk_slot,

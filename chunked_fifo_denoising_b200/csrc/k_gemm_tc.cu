@@ -228,6 +228,70 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + half * HALF;
       if (half * HALF >= BN) {
         // no columns for this warp group
+      } else if (e.rope && n0 < 2 * e.rope_d) {
+        // q or k heads: per-head RMSNorm and rotary positions, head by head
+        const int hd = e.rope_hd;
+        const int grow = row < M ? row : M - 1;  // keep table lookups in range
+        const int ci = grow / e.rows_per_chunk, tk = grow - ci * e.rows_per_chunk;
+        const int fr = tk / (e.rope_Hq * e.rope_Wq);
+        const int py = (tk / e.rope_Wq) % e.rope_Hq, px = tk % e.rope_Wq;
+        const float2* tt = e.rope_t + (long long)(ci * e.rope_Fq + fr) * e.rope_nt;
+        const float2* ty = e.rope_y + (long long)py * e.rope_nh;
+        const float2* tx = e.rope_x + (long long)px * e.rope_nh;
+#pragma unroll 1
+        for (int hb = 0; hb < HALF / hd; ++hb) {
+          const int colh = n0 + hb * hd;
+          const int part = colh >= e.rope_d;
+          const float* wn = (part ? e.k_w : e.q_w) + (colh - part * e.rope_d);
+          // pass 1: sum of squares of the head's biased values
+          float ss = 0.0f;
+#pragma unroll 1
+          for (int i = 0; i < hd / 32; ++i) {
+            float v[32];
+            tmem_ld32(tbase + hb * hd + i * 32, v);
+            add_bias<32>(e, colh + i * 32, N, v);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) ss = fmaf(v[k], v[k], ss);
+          }
+          const float inv = 1.0f / sqrtf(ss / (float)hd + 1e-6f);
+          // pass 2: normalise, scale, rotate each pair, store 64 columns at a time
+#pragma unroll 1
+          for (int g = 0; g < hd / 64; ++g) {
+            const int col0 = colh + g * 64;
+            float v[64];
+            float* v0 = v;
+            tmem_ld32(tbase + hb * hd + g * 64, *reinterpret_cast<float(*)[32]>(v0));
+            tmem_ld32(tbase + hb * hd + g * 64 + 32, *reinterpret_cast<float(*)[32]>(v0 + 32));
+            add_bias<64>(e, col0, N, v);
+            uint32_t w[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const int l = g * 32 + j;  // pair index within the head
+              const float a = v[2 * j] * inv * wn[g * 64 + 2 * j];
+              const float b = v[2 * j + 1] * inv * wn[g * 64 + 2 * j + 1];
+              float2 cs;
+              if (l < e.rope_nt) cs = tt[l];
+              else if (l < e.rope_nt + e.rope_nh) cs = ty[l - e.rope_nt];
+              else cs = tx[l - e.rope_nt - e.rope_nh];
+              w[j] = pack_bf16(a * cs.x - b * cs.y, a * cs.y + b * cs.x);
+            }
+            if (e.cache && row < M && row >= e.cache_row0 && row < e.cache_row0 + e.cache_rows &&
+                col0 >= e.cache_col0) {
+              uint4* d = reinterpret_cast<uint4*>((bf16*)e.cache + (long long)(row - e.cache_row0) * e.ldc +
+                                                  (col0 - e.cache_col0));
+              for (int j = 0; j < 8; ++j) d[j] = make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+            }
+            if (lane == 0) bulk_wait_read<0>();
+            __syncwarp();
+            stage_row(box, lane, w);
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&maps.out, col0, row_base, box);
+              bulk_commit();
+            }
+          }
+        }
       } else if (bf16_out) {
 #pragma unroll 1
         for (int g = 0; g < HALF / 64; ++g) {

@@ -277,6 +277,70 @@ cudaError_t layernorm_mod(const LnParams& p, cudaStream_t s) {
 }
 
 // ---------------------------------------------------------------------------
+// Per-head RMSNorm + 3-D rotary positions of q and k, in place.  One block
+// per row: each thread owns pairs of channels; pass 1 stores every pair's
+// sum of squares in shared memory, pass 2 reduces per head, pass 3 normalises,
+// scales by the per-channel weight and rotates each pair by its angle.
+// ---------------------------------------------------------------------------
+constexpr int RP_THREADS = 256;
+
+template <typename T>
+__global__ void __launch_bounds__(RP_THREADS) qk_norm_rope_kernel(RopeParams p) {
+  extern __shared__ float rp_sm[];  // [d/2] pair sums, then [n_heads] inverse rms
+  float* ss = rp_sm;
+  float* inv = rp_sm + p.d / 2;
+  const int row = blockIdx.x;
+  const int half = p.d / 2;               // pairs per part
+  const int hp = (p.d / p.n_heads) / 2;   // pairs per head
+  const int c = row / p.Lc, t = row - (row / p.Lc) * p.Lc;
+  const int f = t / (p.Hq * p.Wq), y = (t / p.Wq) % p.Hq, x = t % p.Wq;
+  T* base = (T*)p.qkv + (long long)row * p.ld;
+  for (int part = 0; part < 2; ++part) {
+    T* v = base + part * p.d;
+    for (int i = threadIdx.x; i < half; i += RP_THREADS) {
+      const float a = to_f(v[2 * i]), b = to_f(v[2 * i + 1]);
+      ss[i] = a * a + b * b;
+    }
+    __syncthreads();
+    for (int h = threadIdx.x; h < p.n_heads; h += RP_THREADS) {
+      float acc = 0.0f;
+      for (int i = 0; i < hp; ++i) acc += ss[h * hp + i];
+      inv[h] = 1.0f / sqrtf(acc / (float)(2 * hp) + 1e-6f);
+    }
+    __syncthreads();
+    const float* w = part ? p.k_w : p.q_w;
+    for (int i = threadIdx.x; i < half; i += RP_THREADS) {
+      const int h = i / hp, l = i - (i / hp) * hp;
+      const float r = inv[h];
+      const float a = to_f(v[2 * i]) * r * w[2 * i];
+      const float b = to_f(v[2 * i + 1]) * r * w[2 * i + 1];
+      float2 cs;
+      if (l < p.nt) cs = p.rope_t[(long long)(c * p.Fq + f) * p.nt + l];
+      else if (l < p.nt + p.nh) cs = p.rope_y[(long long)y * p.nh + (l - p.nt)];
+      else cs = p.rope_x[(long long)x * p.nh + (l - p.nt - p.nh)];
+      const T ra = from_f<T>(a * cs.x - b * cs.y);
+      const T rb = from_f<T>(a * cs.y + b * cs.x);
+      v[2 * i] = ra;
+      v[2 * i + 1] = rb;
+      if (part == 1 && p.cache && row < p.Lc) {
+        T* cr = (T*)p.cache + (long long)row * p.ldc;
+        cr[2 * i] = ra;
+        cr[2 * i + 1] = rb;
+      }
+    }
+    __syncthreads();
+  }
+}
+
+cudaError_t qk_norm_rope(const RopeParams& p, cudaStream_t s) {
+  if (p.M <= 0) return cudaSuccess;
+  const size_t smem = (size_t)(p.d / 2 + p.n_heads) * sizeof(float);
+  if (p.f32) qk_norm_rope_kernel<float><<<p.M, RP_THREADS, smem, s>>>(p);
+  else qk_norm_rope_kernel<bf16><<<p.M, RP_THREADS, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
 // Patch gather: ring slot [C][F][H][W] -> token rows [Lc][C*pt*ph*pw].
 // One thread per output element; consecutive threads walk the feature index.
 // ---------------------------------------------------------------------------

@@ -93,6 +93,9 @@ struct dp_queue {
   long long Mmax = 0;
   dp::DevBuf ring, x, h, qkv, attn, u, textkv, cache[2], modtab, hmod;
   dp::DevBuf d_sel, d_slot, d_dsig;   // per batch chunk tables (device)
+  dp::DevBuf rope_t, rope_y, rope_x;  // rotary (cos, sin) tables (qk_norm_rope)
+  float* h_rope_t = nullptr;          // pinned staging of the per-step temporal table
+  int rope_Fq = 0, rope_nt = 0, rope_nh = 0;
   int* h_sel = nullptr;               // pinned staging
   int* h_slot = nullptr;
   float* h_dsig = nullptr;

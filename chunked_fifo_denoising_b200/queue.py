@@ -58,7 +58,8 @@ class Model:
             shape.latent_ch, shape.patch_t, shape.patch_h, shape.patch_w, shape.text_len,
             shape.text_in_dim,
             B.DP_PREC_BF16 if precision == "bf16" else B.DP_PREC_FP32_VALIDATE,
-            B.DP_NEIGHBOURS_BOTH if neighbours == "both" else B.DP_NEIGHBOURS_PRED)
+            B.DP_NEIGHBOURS_BOTH if neighbours == "both" else B.DP_NEIGHBOURS_PRED,
+            1 if getattr(shape, "qk_norm_rope", False) else 0)
         self.handle = C.c_void_p()
         B.check(B.dp_model_create(self.cfg, _stream_handle(stream), self.handle), "dp_model_create")
         self.queues = []

@@ -100,6 +100,11 @@ typedef struct {
   int text_in_dim;  /* prompt feature width; != dim adds a projection */
   dp_precision prec;
   dp_neighbours neighbours;
+  int qk_norm_rope;  /* 1: self-attention q and k get a per-head RMSNorm (eps 1e-6,
+                        weights L_QNORM_W / L_KNORM_W) and 3-D rotary positions
+                        (temporal = chunk id * frames + frame, row, column; the
+                        head_dim/2 pairs split into temporal / height / width
+                        bands, height = width = floor(head_dim/6) pairs) */
 } dp_model_config;
 
 /* Queue shape.  One chunk = latent_ch x frames_per_chunk x lat_h x lat_w fp32,
@@ -123,6 +128,7 @@ typedef struct {
  *   L_MOD [6d]  L_QKV_W [3d][d] L_QKV_B [3d]  L_O_W [d][d] L_O_B [d]
  *   L_CQ_W, L_CK_W, L_CV_W, L_CO_W [d][d] with biases [d]
  *   L_FFN1_W [F][d] L_FFN1_B [F]  L_FFN2_W [d][F] L_FFN2_B [d]
+ *   L_QNORM_W [d] L_KNORM_W [d] (only with qk_norm_rope)
  * TEXT_* exist only when text_in_dim != dim. */
 typedef enum {
   DP_PATCH_W = 0, DP_PATCH_B, DP_TEXT_W, DP_TEXT_B,
@@ -131,6 +137,7 @@ typedef enum {
   DP_L_MOD, DP_L_QKV_W, DP_L_QKV_B, DP_L_O_W, DP_L_O_B,
   DP_L_CQ_W, DP_L_CQ_B, DP_L_CK_W, DP_L_CK_B, DP_L_CV_W, DP_L_CV_B,
   DP_L_CO_W, DP_L_CO_B, DP_L_FFN1_W, DP_L_FFN1_B, DP_L_FFN2_W, DP_L_FFN2_B,
+  DP_L_QNORM_W, DP_L_KNORM_W,
   DP_PARAM_COUNT
 } dp_param;
 

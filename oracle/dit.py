@@ -202,6 +202,70 @@ def self_attention_with_predecessor(q, k, v, k_pred, v_pred, n_heads):
 
 
 # ---------------------------------------------------------------------------
+# Per-head QK RMSNorm and 3-D rotary positions (optional block variant)
+# ---------------------------------------------------------------------------
+
+RMS_EPS = 1e-6
+
+
+def rms_norm_heads(x, w, n_heads, eps=RMS_EPS):
+    """Each head's slice of every row divided by its root mean square, then
+    scaled per channel by w (length d).
+
+    reading: the write-up names Wan2.1's DiT without its block; this variant
+    normalises q and k per head (over head_dim) with a learned weight.
+    """
+    L, d = x.shape
+    hd = d // n_heads
+    xh = x.reshape(L, n_heads, hd)
+    r = np.sqrt((xh ** 2).mean(axis=-1, keepdims=True) + eps)
+    return (xh / r).reshape(L, d) * np.asarray(w, np.float64)
+
+
+def rope_bands(hd):
+    """Pairs per axis (temporal, height, width) of a head of hd channels:
+    h = w = floor(hd / 6), t = hd / 2 - 2 h."""
+    nh = (hd // 2) // 3
+    return hd // 2 - 2 * nh, nh, nh
+
+
+def rope_angles(pos_t, pos_y, pos_x, hd, base=10000.0):
+    """Rotation angle of every pair of a head for each token.
+
+    reading: rotary embedding (Su et al., 2021) on interleaved pairs
+    (x_{2i}, x_{2i+1}); the hd/2 pairs are split into a temporal, a height and
+    a width band; pair l of a band of n pairs turns by pos * base^(-l / n).
+    Positions are absolute: the temporal one is chunk id * frames per chunk +
+    frame, so a chunk and its persisted neighbour keep their offset.
+    """
+    nt, nh, nw = rope_bands(hd)
+    cols = []
+    for pos, n in ((pos_t, nt), (pos_y, nh), (pos_x, nw)):
+        theta = np.power(base, -np.arange(n, dtype=np.float64) / n)
+        cols.append(np.outer(np.asarray(pos, np.float64), theta))
+    return np.concatenate(cols, axis=1)   # [tokens][hd/2]
+
+
+def apply_rope(x, angles, n_heads):
+    """Rotates every pair (x_{2i}, x_{2i+1}) of every head by angles[:, i]."""
+    L, d = x.shape
+    hd = d // n_heads
+    xh = x.reshape(L, n_heads, hd // 2, 2)
+    c = np.cos(angles)[:, None, :]
+    s = np.sin(angles)[:, None, :]
+    a, b = xh[..., 0], xh[..., 1]
+    out = np.stack([a * c - b * s, a * s + b * c], axis=-1)
+    return out.reshape(L, d)
+
+
+def token_positions(chunk_id, F, H, W, pt, ph, pw):
+    """(t, y, x) of every token of a chunk, in patchify order."""
+    Fq, Hq, Wq = F // pt, H // ph, W // pw
+    f, y, x = np.meshgrid(np.arange(Fq), np.arange(Hq), np.arange(Wq), indexing="ij")
+    return (chunk_id * Fq + f).ravel(), y.ravel(), x.ravel()
+
+
+# ---------------------------------------------------------------------------
 # Text
 # ---------------------------------------------------------------------------
 
@@ -264,6 +328,10 @@ def velocity(latents, levels, chunk_ids, pred_kv, p, tkv, shape, T, use_pred=Tru
     C, F, Hh, W = latents[0].shape
     x = [linear(patchify(np.asarray(l, np.float64), m.patch_t, m.patch_h, m.patch_w),
                 p["patch.w"], p["patch.b"]) for l in latents]
+    rope = getattr(m, "qk_norm_rope", False)
+    if rope:
+        ang = [rope_angles(*token_positions(k, F, Hh, W, m.patch_t, m.patch_h, m.patch_w), d // H)
+               for k in chunk_ids]
     mods = [level_modulation(j, T, p, m.freq_dim) for j in levels]
     kept = [] if keep_kv_of is not None else None
     for l in range(m.n_layers):
@@ -273,8 +341,12 @@ def velocity(latents, levels, chunk_ids, pred_kv, p, tkv, shape, T, use_pred=Tru
             sh_a, sc_a, g_a, sh_f, sc_f, g_f = split_mod(mods[i][0] + tab, d)
             h = modulate(layer_norm(x[i]), sh_a, sc_a)
             qkv = linear(h, p["layer.qkv.w"][l], p["layer.qkv.b"][l])
-            q.append(qkv[:, :d])
-            k.append(qkv[:, d:2 * d])
+            qi, ki = qkv[:, :d], qkv[:, d:2 * d]
+            if rope:
+                qi = apply_rope(rms_norm_heads(qi, p["layer.qnorm.w"][l], H), ang[i], H)
+                ki = apply_rope(rms_norm_heads(ki, p["layer.knorm.w"][l], H), ang[i], H)
+            q.append(qi)
+            k.append(ki)
             v.append(qkv[:, 2 * d:])
         if kept is not None:
             kept.append((k[keep_kv_of].copy(), v[keep_kv_of].copy()))

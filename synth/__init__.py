@@ -119,6 +119,7 @@ class ModelShape:
     patch_t: int = 1
     patch_h: int = 2
     patch_w: int = 2
+    qk_norm_rope: bool = False   # per-head RMSNorm of q, k and 3-D rotary positions
 
     @property
     def head_dim(self) -> int:
@@ -200,6 +201,11 @@ def truncated(w: Workload, n_layers: int) -> Workload:
     return dataclasses.replace(w, model=dataclasses.replace(w.model, n_layers=n_layers))
 
 
+def with_qk_norm_rope(w: Workload) -> Workload:
+    """The same workload with per-head QK RMSNorm and 3-D rotary positions."""
+    return dataclasses.replace(w, model=dataclasses.replace(w.model, qk_norm_rope=True))
+
+
 # --------------------------------------------------------------------------
 # Parameter inventory: (name, shape, per_layer).  Linear weights are stored
 # [out][in] row-major.  Tensor id ``a`` of a parameter is its index here.
@@ -243,10 +249,12 @@ def param_specs(m: ModelShape):
         ("layer.ffn2.w", (d, F), True),
         ("layer.ffn2.b", (d,), True),
     ]
+    if m.qk_norm_rope:
+        specs += [("layer.qnorm.w", (d,), True), ("layer.knorm.w", (d,), True)]
     return specs
 
 
-ALL_PARAM_NAMES = [s[0] for s in param_specs(ModelShape(1, 8, 1, 8, 8, 1, 16))]
+ALL_PARAM_NAMES = [s[0] for s in param_specs(ModelShape(1, 8, 1, 8, 8, 1, 16, qk_norm_rope=True))]
 
 
 def param_tensor_id(name: str) -> int:
@@ -257,15 +265,18 @@ WEIGHT_STD = 0.02
 
 
 def make_params(m: ModelShape, seed: int = SEED_WEIGHTS, std: float = WEIGHT_STD):
-    """Every parameter ~ N(0, std^2), float32.  Per-layer ones are lists."""
+    """Every parameter ~ N(0, std^2), float32, except the RMSNorm weights
+    (names ending in "norm.w"), which are 1 + N(0, std^2).  Per-layer ones are
+    lists."""
     out = {}
     for name, shape, per_layer in param_specs(m):
         a = param_tensor_id(name)
         n = int(np.prod(shape))
+        mean = np.float32(1.0) if name.endswith("norm.w") else np.float32(0.0)
         if per_layer:
-            out[name] = [normal(seed, a, l, n, std).reshape(shape) for l in range(m.n_layers)]
+            out[name] = [normal(seed, a, l, n, std).reshape(shape) + mean for l in range(m.n_layers)]
         else:
-            out[name] = normal(seed, a, 0, n, std).reshape(shape)
+            out[name] = normal(seed, a, 0, n, std).reshape(shape) + mean
     return out
 
 

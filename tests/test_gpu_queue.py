@@ -8,7 +8,7 @@ float64 oracle on identical seeded inputs:
 * bf16 production mode: one queue step from the same state within relative L2
   2e-2 on the velocity of every chunk, on the persisted K/V and on the latents
   (small workload; Wan-1.3B shapes with two layers; Wan-14B shapes with one
-  layer);
+  layer; the bidirectional neighbourhood; QK RMSNorm with rotary positions);
 * resuming from latents and persisted K/V read mid-stream is bit-exact;
 * error codes, the internal noise generator, flat device memory.
 """
@@ -51,9 +51,11 @@ def make(w, precision, params=None, text=None, n_chunks=None, T=None, ready=2, n
     return model, queue, params, text
 
 
-@pytest.mark.parametrize("neighbours", ["pred", "both"])
-def test_tiny_fp32_stream_matches_oracle(neighbours):
+@pytest.mark.parametrize("neighbours,rope", [("pred", False), ("both", False), ("pred", True)])
+def test_tiny_fp32_stream_matches_oracle(neighbours, rope):
     w = synth.WORKLOADS["tiny_fp32"]
+    if rope:
+        w = synth.with_qk_norm_rope(w)
     m, q = w.model, w.queue
     model, queue, p, text = make(w, "fp32", neighbours=neighbours)
     noise = [synth.make_noise(m, q, k) for k in range(q.n_chunks)]
@@ -169,6 +171,12 @@ def test_bf16_step_small():
 def test_bf16_step_small_bidirectional():
     """The bidirectional neighbourhood: chunk k also reads chunk k+1's K/V."""
     _one_step_parity(synth.WORKLOADS["small_bf16"], neighbours="both")
+
+
+def test_bf16_step_small_qk_norm_rope():
+    """Per-head QK RMSNorm and 3-D rotary positions; the persisted K of the
+    head chunk is the rotated one."""
+    _one_step_parity(synth.with_qk_norm_rope(synth.WORKLOADS["small_bf16"]))
 
 
 def test_bf16_step_wan13b_shapes_two_layers():

@@ -448,3 +448,91 @@ def test_bidirectional_link_reaches_both_ways(tiny):
     w0, _ = fp(lat, lv, ids, None, None)
     w1, _ = fp(lat2, lv, ids, None, None)
     assert np.array_equal(w0[0], w1[0]) and np.array_equal(w0[1], w1[1])
+
+
+# ---------------------------------------------------------------------------
+# per-head QK RMSNorm and 3-D rotary positions
+# ---------------------------------------------------------------------------
+
+def test_rms_norm_heads_closed_form():
+    rng = np.random.default_rng(10)
+    x = rng.normal(2.0, 3.0, size=(5, 16))
+    y = dit.rms_norm_heads(x, np.ones(16), 4, eps=0.0)
+    assert np.allclose((y.reshape(5, 4, 4) ** 2).mean(-1), 1.0)
+    # per head: scaling one head's slice leaves the other heads unchanged
+    x2 = x.copy(); x2[:, 4:8] *= 7.0
+    y2 = dit.rms_norm_heads(x2, np.ones(16), 4, eps=0.0)
+    assert np.allclose(y, y2)
+    w = rng.normal(size=16)
+    assert np.allclose(dit.rms_norm_heads(x, w, 4), dit.rms_norm_heads(x, np.ones(16), 4) * w)
+
+
+def test_rope_bands_and_rotation():
+    assert dit.rope_bands(128) == (22, 21, 21)
+    assert dit.rope_bands(64) == (12, 10, 10)
+    assert dit.rope_bands(16) == (4, 2, 2)
+    rng = np.random.default_rng(11)
+    x = rng.normal(size=(6, 32))
+    t, y, xx = rng.integers(0, 50, 6), rng.integers(0, 30, 6), rng.integers(0, 52, 6)
+    ang = dit.rope_angles(t, y, xx, 16)
+    r = dit.apply_rope(x, ang, 2)
+    # rotation: every pair keeps its length
+    assert np.allclose(np.hypot(r[:, 0::2], r[:, 1::2]), np.hypot(x[:, 0::2], x[:, 1::2]))
+    # position zero is the identity; a hand example: pair 0 of the temporal band
+    # turns by t radians (base^0 = 1)
+    assert np.allclose(dit.apply_rope(x, dit.rope_angles(np.zeros(6), np.zeros(6), np.zeros(6), 16), 2), x)
+    one = np.zeros((1, 16)); one[0, 0] = 1.0
+    got = dit.apply_rope(one, dit.rope_angles([2.0], [0.0], [0.0], 16), 1)
+    assert np.allclose(got[0, :2], [math.cos(2.0), math.sin(2.0)])
+    # the last temporal pair of hd = 16 (band of 4) turns by t * 10000^(-3/4)
+    one = np.zeros((1, 16)); one[0, 6] = 1.0
+    got = dit.apply_rope(one, dit.rope_angles([3.0], [0.0], [0.0], 16), 1)
+    a = 3.0 * 10000.0 ** (-3 / 4)
+    assert np.allclose(got[0, 6:8], [math.cos(a), math.sin(a)])
+
+
+def test_rope_scores_depend_on_relative_position_only():
+    """q(p1) . k(p2) after rotation is a function of p1 - p2: shifting every
+    position by the same offset leaves attention unchanged."""
+    rng = np.random.default_rng(12)
+    q, k, v = rng.normal(size=(5, 32)), rng.normal(size=(7, 32)), rng.normal(size=(7, 32))
+    pq = [rng.integers(0, 40, 5) for _ in range(3)]
+    pk = [rng.integers(0, 40, 7) for _ in range(3)]
+    o1 = dit.attention(dit.apply_rope(q, dit.rope_angles(*pq, 16), 2),
+                       dit.apply_rope(k, dit.rope_angles(*pk, 16), 2), v, 2)
+    shift = (1000, 17, 5)
+    o2 = dit.attention(dit.apply_rope(q, dit.rope_angles(*[a + s for a, s in zip(pq, shift)], 16), 2),
+                       dit.apply_rope(k, dit.rope_angles(*[a + s for a, s in zip(pk, shift)], 16), 2), v, 2)
+    assert np.allclose(o1, o2, atol=1e-10)
+
+
+def test_token_positions_follow_patch_order():
+    t, y, x = dit.token_positions(3, 2, 4, 6, 1, 2, 2)
+    assert len(t) == 2 * 2 * 3
+    # token index (f=1, row=1, col=2) = (1 * 2 + 1) * 3 + 2
+    i = (1 * 2 + 1) * 3 + 2
+    assert (t[i], y[i], x[i]) == (3 * 2 + 1, 1, 2)
+
+
+def test_rope_model_shift_invariance_over_chunk_ids(tiny):
+    """With rotary positions the velocity of a batch does not depend on the
+    absolute chunk ids, only on their offsets (relative positions)."""
+    p, text, noise = tiny
+    m = dataclasses_replace_rope(W.model)
+    q = synth.make_params(m)
+    fn = dit.make_velocity_fn(q, text, m, T=6)
+    lat = [np.asarray(noise[k], np.float64) for k in range(3)]
+    va, _ = fn(lat, [2, 3, 4], [0, 1, 2], None, None)
+    vb, _ = fn(lat, [2, 3, 4], [40, 41, 42], None, None)
+    for a, b in zip(va, vb):
+        assert np.allclose(a, b, atol=1e-10)
+    # and it does depend on the positions: swapping in a non-contiguous layout
+    # of frames is visible (rotary positions are active)
+    fn0 = dit.make_velocity_fn(p, text, W.model, T=6)
+    v0, _ = fn0(lat, [2, 3, 4], [0, 1, 2], None, None)
+    assert not np.allclose(v0[1], va[1])
+
+
+def dataclasses_replace_rope(m):
+    import dataclasses
+    return dataclasses.replace(m, qk_norm_rope=True)
