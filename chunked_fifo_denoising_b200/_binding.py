@@ -49,7 +49,7 @@ class dp_model_config(C.Structure):
 class dp_queue_config(C.Structure):
     _fields_ = [("T", C.c_int), ("frames_per_chunk", C.c_int), ("lat_h", C.c_int),
                 ("lat_w", C.c_int), ("n_chunks", C.c_longlong), ("ready_capacity", C.c_int),
-                ("seed", C.c_ulonglong)]
+                ("seed", C.c_ulonglong), ("noise_mode", C.c_int)]
 
 
 class dp_queue_info(C.Structure):
@@ -96,6 +96,7 @@ _SIGS = {
     "dp_queue_step": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int]),
     "dp_queue_pop": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.POINTER(C.c_longlong)]),
     "dp_queue_close": (C.c_int, [C.c_void_p]),
+    "dp_queue_set_noise_pool": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int]),
     "dp_queue_sync": (C.c_int, [C.c_void_p]),
     "dp_queue_inspect": (C.c_int, [C.c_void_p, C.POINTER(dp_queue_info), C.c_void_p, C.c_void_p,
                                    C.c_void_p, C.c_void_p, C.c_int]),
@@ -164,6 +165,7 @@ def dp_queue_init(m, qc, text, loc, out): return _call("dp_queue_init", m, C.byr
 def dp_queue_step(q, noise, loc): return _call("dp_queue_step", q, noise, loc)
 def dp_queue_pop(q, out, loc, cid): return _call("dp_queue_pop", q, out, loc, C.byref(cid))
 def dp_queue_close(q): return _call("dp_queue_close", q)
+def dp_queue_set_noise_pool(q, pool, loc): return _call("dp_queue_set_noise_pool", q, pool, loc)
 def dp_queue_sync(q): return _call("dp_queue_sync", q)
 def dp_queue_inspect(q, info, ids, levels, slots, positions, cap): return _call("dp_queue_inspect", q, C.byref(info), ids, levels, slots, positions, cap)
 def dp_queue_read_latents(q, out, n, loc): return _call("dp_queue_read_latents", q, out, n, loc)

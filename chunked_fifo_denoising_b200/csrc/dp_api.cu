@@ -316,7 +316,41 @@ dp_status dp_model_set_param(dp_model* m, dp_param id, int layer, const float* s
 namespace {
 
 const int kPredNone = 0, kPredCache = 2;
-const unsigned long long kNoiseTensorId = 1001;  // tensor id of chunk noise in the generator
+const unsigned long long kNoiseTensorId = 1001;    // tensor id of chunk noise in the generator
+const unsigned long long kShuffleTensorId = 1002;  // draws of the coordinated-noise order
+const unsigned long long kPoolTensorId = 1003;     // coordinated-noise pool frames
+
+// SplitMix64 (Steele, Lea, Flood 2014): finaliser and keyed stream draws.
+unsigned long long sm64_mix(unsigned long long z) {
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  return z ^ (z >> 31);
+}
+unsigned long long sm64_key(unsigned long long seed, unsigned long long a, unsigned long long b) {
+  const unsigned long long g = 0x9E3779B97F4A7C15ull;
+  unsigned long long k = sm64_mix((seed + 1) * g);
+  k = sm64_mix(k + (a + 1) * g);
+  return sm64_mix(k + (b + 1) * g);
+}
+
+// Pool frames of chunk k (coordinated noise): the F frames chunk k-1 does not
+// use, 0..F-1 for even k and F..2F-1 for odd k, shuffled by Fisher-Yates with
+// the draws of stream (seed, 1002, k): for i = F-1 .. 1 swap i with draw mod (i+1).
+PoolGather coordinated_frames(unsigned long long seed, long long k, int F) {
+  PoolGather g;
+  const int base = (k % 2 == 0) ? 0 : F;
+  for (int f = 0; f < F; ++f) g.src[f] = base + f;
+  const unsigned long long key = sm64_key(seed, kShuffleTensorId, (unsigned long long)k);
+  unsigned long long t = 0;
+  for (int i = F - 1; i >= 1; --i, ++t) {
+    const unsigned long long draw = sm64_mix(key + (t + 1) * 0x9E3779B97F4A7C15ull);
+    const int j = (int)(draw % (unsigned long long)(i + 1));
+    const int tmp = g.src[i];
+    g.src[i] = g.src[j];
+    g.src[j] = tmp;
+  }
+  return g;
+}
 
 struct Plan {
   bool push = false;
@@ -691,7 +725,7 @@ static dp_status upload_tables(dp_queue* q, const Plan& pl) {
 static void free_queue(dp_queue* q) {
   DevBuf* bufs[] = {&q->ring, &q->x, &q->h, &q->qkv, &q->attn, &q->u, &q->textkv, &q->cache[0],
                     &q->cache[1], &q->modtab, &q->hmod, &q->d_sel, &q->d_slot, &q->d_dsig,
-                    &q->rope_t, &q->rope_y, &q->rope_x};
+                    &q->rope_t, &q->rope_y, &q->rope_x, &q->noise_pool};
   for (DevBuf* b : bufs) dev_free(*b);
   if (q->h_rope_t) cudaFreeHost(q->h_rope_t);
   if (q->h_sel) cudaFreeHost(q->h_sel);
@@ -786,6 +820,9 @@ dp_status dp_queue_init(dp_model* m, const dp_queue_config* qc, const float* tex
       qc->lat_h % c.patch_h || qc->lat_w < 1 || qc->lat_w % c.patch_w)
     return fail(DP_ERR_INVALID_ARG, "chunk shape not divisible by the patch size");
   if (qc->n_chunks == 0 || qc->n_chunks < -1) return fail(DP_ERR_INVALID_ARG, "n_chunks must be > 0 or -1");
+  if (qc->noise_mode != 0 && qc->noise_mode != 1) return fail(DP_ERR_INVALID_ARG, "bad noise_mode");
+  if (qc->noise_mode == 1 && qc->frames_per_chunk > 64)
+    return fail(DP_ERR_INVALID_ARG, "coordinated noise supports at most 64 frames per chunk");
   if (text_loc != DP_LOC_DEVICE && text_loc != DP_LOC_HOST) return fail(DP_ERR_INVALID_ARG, "bad location");
   for (int i = 0; i < DP_PARAM_COUNT; ++i)
     for (char sset : m->params[i].set)
@@ -823,6 +860,7 @@ dp_status dp_queue_init(dp_model* m, const dp_queue_config* qc, const float* tex
   QA(q->d_sel, (size_t)qc->T * 4, "chunk levels");
   QA(q->d_slot, (size_t)qc->T * 4, "chunk slots");
   QA(q->d_dsig, (size_t)qc->T * 4, "chunk sigma steps");
+  if (qc->noise_mode == 1) QA(q->noise_pool, (size_t)2 * q->chunk_numel * 4, "noise pool");
   if (c.qk_norm_rope) {
     q->rope_Fq = qc->frames_per_chunk / c.patch_t;
     q->rope_nh = (m->hd / 2) / 3;
@@ -843,6 +881,16 @@ dp_status dp_queue_init(dp_model* m, const dp_queue_config* qc, const float* tex
     if (e != cudaSuccess) s = fail(DP_ERR_OOM, "pinned staging: %s", cudaGetErrorString(e));
   }
   if (s == DP_OK) s = build_tables(q, text, text_loc);
+  if (s == DP_OK && qc->noise_mode == 1) {
+    // default pool: 2F frames of N(0,1), frame b from stream (seed, 1003, b)
+    const long long fe = (long long)c.latent_ch * qc->lat_h * qc->lat_w;
+    for (int b = 0; b < 2 * qc->frames_per_chunk && s == DP_OK; ++b) {
+      cudaError_t e = normal_fill(qc->seed, kPoolTensorId, (unsigned long long)b,
+                                  q->noise_pool.as<float>() + (size_t)b * fe, fe, m->stream);
+      if (e == cudaSuccess) e = cudaStreamSynchronize(m->stream);
+      if (e != cudaSuccess) s = fail(DP_ERR_CUDA, "noise pool: %s", cudaGetErrorString(e));
+    }
+  }
   if (s == DP_OK && c.qk_norm_rope) {
     // row and column rotary tables, fixed for the queue: angle = pos * 10000^(-l/nh)
     const int nh = q->rope_nh;
@@ -889,6 +937,11 @@ dp_status dp_queue_step(dp_queue* q, const float* noise, dp_loc loc) {
     if (noise) {
       DP_CK(cudaMemcpyAsync(slot, noise, (size_t)q->chunk_numel * 4,
                             loc == DP_LOC_HOST ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice, s));
+    } else if (q->qc.noise_mode == 1) {
+      const int F = q->qc.frames_per_chunk;
+      DP_CK(noise_from_pool(q->noise_pool.as<float>(), m->cfg.latent_ch, F,
+                            (long long)q->qc.lat_h * q->qc.lat_w,
+                            coordinated_frames(q->qc.seed, q->next_id, F), slot, s));
     } else {
       DP_CK(normal_fill(q->qc.seed, kNoiseTensorId, (unsigned long long)q->next_id, slot,
                         q->chunk_numel, s));
@@ -926,6 +979,18 @@ dp_status dp_queue_pop(dp_queue* q, float* out, dp_loc loc, long long* chunk_id)
   if (loc == DP_LOC_HOST) DP_CK(cudaStreamSynchronize(s));
   if (chunk_id) *chunk_id = q->ready_lo;
   q->ready_lo += 1;
+  return DP_OK;
+}
+
+dp_status dp_queue_set_noise_pool(dp_queue* q, const float* pool, dp_loc loc) {
+  clear_error();
+  if (!q || !pool) return fail(DP_ERR_INVALID_ARG, "NULL argument");
+  if (q->qc.noise_mode != 1) return fail(DP_ERR_STATE, "the queue does not use coordinated noise");
+  if (loc != DP_LOC_DEVICE && loc != DP_LOC_HOST) return fail(DP_ERR_INVALID_ARG, "bad location");
+  DP_CK(cudaMemcpyAsync(q->noise_pool.p, pool, (size_t)2 * q->chunk_numel * 4,
+                        loc == DP_LOC_HOST ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice,
+                        q->m->stream));
+  DP_CK(cudaStreamSynchronize(q->m->stream));
   return DP_OK;
 }
 

@@ -116,6 +116,11 @@ cudaError_t normal_fill(unsigned long long seed, unsigned long long a, unsigned 
 // Device status word of kernels launched from the single-kernel entry points.
 int* op_status_word();
 
+// slot [C][F][HW] <- pool [2F][C][HW]: frame f of the chunk is pool frame src[f]
+struct PoolGather { int src[64]; };
+cudaError_t noise_from_pool(const float* pool, int C, int F, long long hw, PoolGather src,
+                            float* slot, cudaStream_t s);
+
 cudaError_t convert_f32_to_bf16(const float* in, bf16* out, long long n, cudaStream_t s);
 cudaError_t convert_bf16_to_f32(const bf16* in, float* out, long long n, cudaStream_t s);
 // strided 2-D copy/convert of a [rows][cols] block between float/bf16 buffers

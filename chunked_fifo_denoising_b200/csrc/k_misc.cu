@@ -464,6 +464,25 @@ cudaError_t normal_fill(unsigned long long seed, unsigned long long a, unsigned 
   return cudaGetLastError();
 }
 
+// Coordinated noise: frames of the new chunk gathered from the noise pool.
+__global__ void pool_gather_kernel(const float* __restrict__ pool, int C, int F, long long hw,
+                                   PoolGather src, float* __restrict__ slot) {
+  const long long total = (long long)C * F * hw;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long e = i % hw;
+    const int f = (int)((i / hw) % F);
+    const int c = (int)(i / (hw * F));
+    slot[i] = pool[((long long)src.src[f] * C + c) * hw + e];
+  }
+}
+
+cudaError_t noise_from_pool(const float* pool, int C, int F, long long hw, PoolGather src,
+                            float* slot, cudaStream_t s) {
+  pool_gather_kernel<<<148 * 4, 256, 0, s>>>(pool, C, F, hw, src, slot);
+  return cudaGetLastError();
+}
+
 // ---------------------------------------------------------------------------
 // Conversions
 // ---------------------------------------------------------------------------

@@ -96,6 +96,7 @@ struct dp_queue {
   dp::DevBuf rope_t, rope_y, rope_x;  // rotary (cos, sin) tables (qk_norm_rope)
   float* h_rope_t = nullptr;          // pinned staging of the per-step temporal table
   int rope_Fq = 0, rope_nt = 0, rope_nh = 0;
+  dp::DevBuf noise_pool;              // [2F][C][H][W] (noise_mode 1)
   int* h_sel = nullptr;               // pinned staging
   int* h_slot = nullptr;
   float* h_dsig = nullptr;

@@ -102,9 +102,10 @@ class Queue:
     """A FIFO denoising queue of ``T`` levels on a model."""
 
     def __init__(self, model, text, T, frames_per_chunk, lat_h, lat_w, n_chunks=-1,
-                 ready_capacity=2, seed=3):
+                 ready_capacity=2, seed=3, noise="fresh"):
         self.model = model
-        self.qc = B.dp_queue_config(T, frames_per_chunk, lat_h, lat_w, n_chunks, ready_capacity, seed)
+        self.qc = B.dp_queue_config(T, frames_per_chunk, lat_h, lat_w, n_chunks, ready_capacity, seed,
+                                    1 if noise == "coordinated" else 0)
         s = model.shape
         self.chunk_shape = (s.latent_ch, frames_per_chunk, lat_h, lat_w)
         self.chunk_numel = int(np.prod(self.chunk_shape))
@@ -134,6 +135,10 @@ class Queue:
         cid = C.c_longlong(-1)
         st = B.dp_queue_pop(self.handle, p, loc, cid)
         return st, cid.value
+
+    def set_noise_pool(self, pool):
+        p, loc = _ptr(pool)
+        B.check(B.dp_queue_set_noise_pool(self.handle, p, loc), "dp_queue_set_noise_pool")
 
     def close_stream(self):
         B.check(B.dp_queue_close(self.handle), "dp_queue_close")

@@ -116,6 +116,12 @@ typedef struct {
   long long n_chunks;     /* chunks in the stream; -1 = until dp_queue_close */
   int ready_capacity;     /* clean chunks that may wait for dp_queue_pop (>=1) */
   unsigned long long seed;/* seed of the internal noise generator           */
+  int noise_mode;         /* initial latent of a chunk pushed without caller
+                             noise: 0 = fresh N(0,1) per chunk; 1 = coordinated:
+                             from a pool of 2F noise frames, the F frames the
+                             previous chunk did not use (frames 0..F-1 for even
+                             chunk ids, F..2F-1 for odd), in a Fisher-Yates order
+                             driven by SplitMix64 stream (seed, 1002, chunk id) */
 } dp_queue_config;
 
 /* Parameters.  Linear weights are [out][in] row-major fp32; biases [out].
@@ -188,6 +194,11 @@ DP_API dp_status dp_queue_step(dp_queue* q, const float* new_chunk_noise, dp_loc
  * frees its slot; `chunk_id` (may be NULL) receives its id.  Chunk ids pop in
  * strictly increasing order.  DP_ERR_EMPTY if none is ready. */
 DP_API dp_status dp_queue_pop(dp_queue* q, float* out, dp_loc loc, long long* chunk_id);
+
+/* Replaces the coordinated-noise pool (noise_mode 1) with `pool`
+ * ([2F][C][H][W] fp32 at `loc`).  By default the pool is drawn N(0,1) on the
+ * device at dp_queue_init (frame b from stream (seed, 1003, b)).  Synchronous. */
+DP_API dp_status dp_queue_set_noise_pool(dp_queue* q, const float* pool, dp_loc loc);
 
 /* Ends an unbounded stream: no further chunk is pushed; steps drain the queue. */
 DP_API dp_status dp_queue_close(dp_queue* q);

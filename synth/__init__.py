@@ -46,6 +46,8 @@ SEED_NOISE = 3
 # Tensor ids used as ``a`` in the stream key.
 TID_TEXT = 1000
 TID_NOISE = 1001
+TID_SHUFFLE = 1002      # draws of the coordinated-noise permutation of chunk b
+TID_NOISE_POOL = 1003   # noise pool frame b (coordinated noise)
 
 
 def _mix64_int(z: int) -> int:
@@ -283,6 +285,13 @@ def make_params(m: ModelShape, seed: int = SEED_WEIGHTS, std: float = WEIGHT_STD
 def make_text(m: ModelShape, seed: int = SEED_TEXT) -> np.ndarray:
     return normal(seed, TID_TEXT, 0, m.text_len * m.text_in_dim).reshape(
         m.text_len, m.text_in_dim)
+
+
+def make_noise_pool(m: ModelShape, q: QueueShape, seed: int = SEED_NOISE) -> np.ndarray:
+    """2F latent frames of N(0,1) noise, [2F][C][H][W]; frame b from stream b."""
+    n = m.latent_ch * q.lat_h * q.lat_w
+    return np.stack([normal(seed, TID_NOISE_POOL, b, n).reshape(m.latent_ch, q.lat_h, q.lat_w)
+                     for b in range(2 * q.frames_per_chunk)])
 
 
 def make_noise(m: ModelShape, q: QueueShape, chunk_id: int, seed: int = SEED_NOISE) -> np.ndarray:

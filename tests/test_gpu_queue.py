@@ -273,6 +273,35 @@ def test_internal_generator_matches_seeded_noise():
     model.close()
 
 
+def test_coordinated_noise_pushes_the_oracle_frames():
+    """noise_mode 1: each pushed chunk is the oracle's selection and order of
+    the pool frames (bit-exact with the pool uploaded); the default pool is the
+    seeded N(0,1) frames of the device generator."""
+    from chunked_fifo_denoising_b200 import Model, Queue
+    from oracle import noise
+    w = synth.WORKLOADS["tiny_fp32"]
+    m, q = w.model, w.queue
+    p = synth.make_params(m)
+    p["out.w"] = np.zeros_like(p["out.w"])   # zero velocity: the latents stay as pushed
+    p["out.b"] = np.zeros_like(p["out.b"])
+    model = Model(m, "fp32")
+    model.set_params(p)
+    text = synth.make_text(m)
+    pool = synth.make_noise_pool(m, q).astype(np.float32)
+    qa = Queue(model, text, 6, q.frames_per_chunk, q.lat_h, q.lat_w, 6, seed=5, noise="coordinated")
+    qa.set_noise_pool(pool)
+    for k in range(5):
+        qa.step(None)
+        lat = qa.read_latents(k + 1)
+        assert np.array_equal(lat[-1], noise.coordinated_noise(pool, k, 5).astype(np.float32)), k
+    qb = Queue(model, text, 6, q.frames_per_chunk, q.lat_h, q.lat_w, 6, seed=3, noise="coordinated")
+    qb.step(None)
+    got = qb.read_latents(1)[0]
+    ref = noise.coordinated_noise(synth.make_noise_pool(m, q, seed=3), 0, 3)
+    assert np.allclose(got, ref, rtol=1e-6, atol=1e-6)
+    model.close()
+
+
 def test_device_memory_flat_in_stream_length():
     """Long-stream workload: memory after init is the same for 32, 64 and 128
     chunks and the steps allocate nothing (two-layer model, zero weights)."""

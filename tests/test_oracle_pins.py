@@ -536,3 +536,42 @@ def test_rope_model_shift_invariance_over_chunk_ids(tiny):
 def dataclasses_replace_rope(m):
     import dataclasses
     return dataclasses.replace(m, qk_norm_rope=True)
+
+
+# ---------------------------------------------------------------------------
+# coordinated noise initialisation
+# ---------------------------------------------------------------------------
+
+def test_coordinated_noise_sets_alternate_and_cover_the_pool():
+    from oracle import noise
+    F = 4
+    for k in range(20):
+        a, b = noise.chunk_frames(k, F, 3), noise.chunk_frames(k + 1, F, 3)
+        assert sorted(a) == list(range(0, F) if k % 2 == 0 else range(F, 2 * F))
+        assert not set(a) & set(b)                     # no repeat between neighbours
+        assert sorted(a + b) == list(range(2 * F))     # together the whole pool
+
+
+def test_coordinated_noise_shuffle_is_a_uniform_permutation():
+    from oracle import noise
+    F = 3
+    counts = np.zeros((F, F))
+    perms = set()
+    for k in range(0, 6000, 2):
+        fr = noise.chunk_frames(k, F, 7)
+        perms.add(tuple(fr))
+        for pos, b in enumerate(fr):
+            counts[pos, b] += 1
+    assert len(perms) == 6                             # every order of 3 frames occurs
+    assert np.allclose(counts / counts.sum(axis=1, keepdims=True), 1 / F, atol=0.04)
+
+
+def test_coordinated_noise_gathers_pool_frames():
+    from oracle import noise
+    rng = np.random.default_rng(13)
+    pool = rng.normal(size=(4, 3, 2, 5))               # 2F = 4 frames, C=3, H=2, W=5
+    lat = noise.coordinated_noise(pool, 1, 3)
+    fr = noise.chunk_frames(1, 2, 3)
+    assert lat.shape == (3, 2, 2, 5)
+    for f in range(2):
+        assert np.array_equal(lat[:, f], pool[fr[f]])
