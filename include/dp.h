@@ -187,7 +187,12 @@ DP_API dp_status dp_queue_init(dp_model* m, const dp_queue_config* qc, const flo
  * x <- x + (sigma_{j-1} - sigma_j) v with sigma_j = j/T, and drops one level;
  * the chunk that reaches level 0 becomes ready for dp_queue_pop.
  * Errors: DP_ERR_FULL (push due, no free slot: pop first), DP_ERR_DRAINED
- * (nothing left to denoise).  On error nothing was enqueued. */
+ * (nothing left to denoise), DP_ERR_STATE (the persisted K/V the head needs
+ * are missing); after these nothing was enqueued and the queue is unchanged.
+ * DP_ERR_CUDA / DP_ERR_INVALID_ARG from a failed launch inside the step leave
+ * part of the step enqueued: the queue must then be destroyed (or reloaded
+ * with dp_queue_load_state).  A queue is not safe to use from several host
+ * threads at once. */
 DP_API dp_status dp_queue_step(dp_queue* q, const float* new_chunk_noise, dp_loc loc);
 
 /* Copies the oldest ready chunk ([C][F][H][W] fp32) to `out` at `loc` and
