@@ -56,6 +56,7 @@ struct AttnParams {
   const void* k0_pred; const void* v0_pred; long long ld_pred; int Lk_pred;
   void* out; long long ldo;
   int succ_in_batch;              // chunk c < n_chunks-1 also reads chunk c+1's own keys
+  int qblocks_per_cta;            // tensor-core path: 256-query blocks per CTA (0 = choose)
 };
 
 struct LnParams {

@@ -10,7 +10,9 @@
 // concatenated.  The same kernel with one shared buffer is the cross-attention
 // to the prompt.
 //
-// CTA = 256 queries (two 128-row tiles A and B) of one (chunk, head), 10 warps:
+// CTA = 256-query blocks (two 128-row tiles A and B each) of one (chunk, head),
+// processed one after the other with TMEM and barriers kept (several blocks
+// per CTA when the key set is short), 10 warps:
 //   warp 0      TMA producer: Q_A, Q_B once; K and V tiles of 128 keys into two
 //               2-stage rings, each tile from whichever buffer it belongs to
 //   warp 1      TMEM owner + MMA issuer, tiles ping-ponged on the tensor core:
@@ -115,17 +117,18 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
   using C = Cfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  __shared__ uint64_t q_full, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2], p_full[2],
-      pv_done[2], done_bar;
+  __shared__ uint64_t q_full, q_empty, k_full[2], k_empty[2], v_full[2], v_empty[2], s_full[2],
+      p_full[2], pv_done[2], done_bar;
   __shared__ uint32_t tmem_base_sh;
   __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y, c = blockIdx.z;
-  const int q0 = blockIdx.x * 2 * BQ;        // first query of tile A within the chunk
-  const bool has_b = q0 + BQ < p.Lq;         // tile B holds at least one query
-  const int qrow0 = c * p.Lq + q0;
-  // key sources of this chunk
+  // this CTA covers 256-query blocks [qb0, qb1) of chunk c, one after the other
+  const int nqb = (p.Lq + 2 * BQ - 1) / (2 * BQ);
+  const int qb0 = blockIdx.x * p.qblocks_per_cta;
+  const int qb1 = min(nqb, qb0 + p.qblocks_per_cta);
+  // key sources of this chunk (the same for every query block)
   int n_p = 0;
   bool pred_cache = false;
   if (c > 0 && p.pred_in_batch) {
@@ -142,6 +145,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
 
   if (threadIdx.x == 0) {
     mbar_init(&q_full, 1);
+    mbar_init(&q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       mbar_init(&k_full[i], 1);
       mbar_init(&k_empty[i], 1);
@@ -168,54 +172,71 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       const int col0 = h * HD;
-      mbar_arrive_expect_tx(&q_full, (has_b ? 2 : 1) * C::T_BYTES);
+      uint32_t issued_k = 0, issued_v = 0, par = 0, q_issued = 0;
+      uint32_t gk = 0;  // K/V tiles issued so far (stage gk & 1, use gk >> 1)
+      bool ok = true;
+      for (int qb = qb0; qb < qb1 && ok; ++qb) {
+        const int bi = qb - qb0;
+        const int q0 = qb * 2 * BQ;
+        const bool has_b = q0 + BQ < p.Lq;
+        const int qrow0 = c * p.Lq + q0;
+        // Q of the previous block is read by its S MMAs only
+        if (bi > 0 && !mbar_wait(&q_empty, (bi - 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
+        mbar_arrive_expect_tx(&q_full, (has_b ? 2 : 1) * C::T_BYTES);
 #pragma unroll
-      for (int s = 0; s < C::NSUB; ++s) {
-        tma_load_2d(smem + C::OFF_QA + s * C::SUB_BYTES, &maps.q, col0 + 64 * s, qrow0, &q_full);
-        if (has_b) tma_load_2d(smem + C::OFF_QB + s * C::SUB_BYTES, &maps.q, col0 + 64 * s, qrow0 + BQ, &q_full);
-      }
-      uint32_t issued_k = 0, issued_v = 0, par = 0;
-      for (int j = 0; j < nt; ++j) {
-        const int st = j & 1;
-        const uint32_t use = (uint32_t)(j >> 1);
-        const CUtensorMap* mk;
-        const CUtensorMap* mv;
-        int row;
-        if (j < tiles_p) {
-          if (pred_cache) {
-            mk = &maps.kp;
-            mv = &maps.vp;
-            row = j * BKV;
-          } else {
+        for (int s = 0; s < C::NSUB; ++s) {
+          tma_load_2d(smem + C::OFF_QA + s * C::SUB_BYTES, &maps.q, col0 + 64 * s, qrow0, &q_full);
+          if (has_b) tma_load_2d(smem + C::OFF_QB + s * C::SUB_BYTES, &maps.q, col0 + 64 * s, qrow0 + BQ, &q_full);
+        }
+        q_issued = bi + 1;
+        for (int j = 0; j < nt; ++j, ++gk) {
+          const int st = gk & 1;
+          const uint32_t use = gk >> 1;
+          const CUtensorMap* mk;
+          const CUtensorMap* mv;
+          int row;
+          if (j < tiles_p) {
+            if (pred_cache) {
+              mk = &maps.kp;
+              mv = &maps.vp;
+              row = j * BKV;
+            } else {
+              mk = &maps.k;
+              mv = &maps.v;
+              row = (int)((c - 1) * p.kv_chunk_rows) + j * BKV;
+            }
+          } else if (j < tiles_p + tiles_o) {
             mk = &maps.k;
             mv = &maps.v;
-            row = (int)((c - 1) * p.kv_chunk_rows) + j * BKV;
+            row = (int)(c * p.kv_chunk_rows) + (j - tiles_p) * BKV;
+          } else {  // successor: chunk c+1's own rows of this batch
+            mk = &maps.k;
+            mv = &maps.v;
+            row = (int)((c + 1) * p.kv_chunk_rows) + (j - tiles_p - tiles_o) * BKV;
           }
-        } else if (j < tiles_p + tiles_o) {
-          mk = &maps.k;
-          mv = &maps.v;
-          row = (int)(c * p.kv_chunk_rows) + (j - tiles_p) * BKV;
-        } else {  // successor: chunk c+1's own rows of this batch
-          mk = &maps.k;
-          mv = &maps.v;
-          row = (int)((c + 1) * p.kv_chunk_rows) + (j - tiles_p - tiles_o) * BKV;
+          if (use > 0 && !mbar_wait(&k_empty[st], (use - 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&k_full[st], C::T_BYTES);
+#pragma unroll
+          for (int s = 0; s < C::NSUB; ++s)
+            tma_load_2d(smem + C::OFF_K + st * C::T_BYTES + s * C::SUB_BYTES, mk, col0 + 64 * s, row, &k_full[st]);
+          issued_k |= 1u << st;
+          par = (par & ~(1u << st)) | ((use & 1u) << st);
+          if (use > 0 && !mbar_wait(&v_empty[st], (use - 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&v_full[st], C::T_BYTES);
+#pragma unroll
+          for (int s = 0; s < C::NSUB; ++s)
+            tma_load_2d(smem + C::OFF_V + st * C::T_BYTES + s * C::SUB_BYTES, mv, col0 + 64 * s, row, &v_full[st]);
+          issued_v |= 1u << st;
         }
-        if (use > 0 && !mbar_wait(&k_empty[st], (use - 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
-        mbar_arrive_expect_tx(&k_full[st], C::T_BYTES);
-#pragma unroll
-        for (int s = 0; s < C::NSUB; ++s)
-          tma_load_2d(smem + C::OFF_K + st * C::T_BYTES + s * C::SUB_BYTES, mk, col0 + 64 * s, row, &k_full[st]);
-        issued_k |= 1u << st;
-        par = (par & ~(1u << st)) | ((use & 1u) << st);
-        if (use > 0 && !mbar_wait(&v_empty[st], (use - 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
-        mbar_arrive_expect_tx(&v_full[st], C::T_BYTES);
-#pragma unroll
-        for (int s = 0; s < C::NSUB; ++s)
-          tma_load_2d(smem + C::OFF_V + st * C::T_BYTES + s * C::SUB_BYTES, mv, col0 + 64 * s, row, &v_full[st]);
-        issued_v |= 1u << st;
       }
       if (abort_flag) {  // let copies in flight land before the CTA exits
-        drain_wait(&q_full, 0);
+        if (q_issued > 0) drain_wait(&q_full, (q_issued - 1) & 1);
         for (int st = 0; st < 2; ++st) {
           if (issued_k & (1u << st)) drain_wait(&k_full[st], (par >> st) & 1u);
           if (issued_v & (1u << st)) drain_wait(&v_full[st], (par >> st) & 1u);
@@ -227,9 +248,9 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
       // ---------------- MMA issuer ----------------
       constexpr uint32_t IDESC_S = idesc_bf16_f32(BQ, BKV, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(BQ, HD, 0, 1);
-      auto issue_s = [&](int X, int j) {
+      auto issue_s = [&](int X, uint32_t g) {
         const uint32_t sQ = smem_u32(smem + (X ? C::OFF_QB : C::OFF_QA));
-        const uint32_t sK = smem_u32(smem + C::OFF_K + (j & 1) * C::T_BYTES);
+        const uint32_t sK = smem_u32(smem + C::OFF_K + (g & 1) * C::T_BYTES);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::SUB_BYTES + (kk & 3) * 32;
@@ -238,43 +259,64 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
         }
         mma_commit(&s_full[X]);
       };
-      auto issue_pv = [&](int X, int j) {
-        const uint32_t sV = smem_u32(smem + C::OFF_V + (j & 1) * C::T_BYTES);
+      auto issue_pv = [&](int X, uint32_t g, int j) {
+        const uint32_t sV = smem_u32(smem + C::OFF_V + (g & 1) * C::T_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk)  // 16 keys = 8 TMEM columns of packed P; 2 atoms of V
           mma_bf16_ts(tmem + C::o_col(X), tmem + C::s_col(X) + kk * 8,
                       desc_sw128(sV + kk * 2048, C::SUB_BYTES, 1024), IDESC_O, (j | kk) != 0);
         mma_commit(&pv_done[X]);
       };
-      bool ok = mbar_wait(&q_full, 0, &abort_flag, status, ST_TIMEOUT_ATTN) &&
-                mbar_wait(&k_full[0], 0, &abort_flag, status, ST_TIMEOUT_ATTN);
-      if (ok) {
+      uint32_t gk = 0;          // K/V tiles consumed so far
+      uint32_t gp[2] = {0, 0};  // P tiles of tile A / tile B consumed so far
+      bool ok = true;
+      for (int qb = qb0; qb < qb1 && ok; ++qb) {
+        const int bi = qb - qb0;
+        const bool has_b = qb * 2 * BQ + BQ < p.Lq;
+        ok = mbar_wait(&q_full, bi & 1, &abort_flag, status, ST_TIMEOUT_ATTN) &&
+             mbar_wait(&k_full[gk & 1], (gk >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN);
+        if (!ok) break;
         tc_fence_after();
-        issue_s(0, 0);
-        if (has_b) issue_s(1, 0);
-        mma_commit(&k_empty[0]);
-      }
-      for (int j = 0; j < nt && ok; ++j) {
-        const bool next = j + 1 < nt;
-        if (!mbar_wait(&v_full[j & 1], (j >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
-        if (!mbar_wait(&p_full[0], j & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
-        tc_fence_after();
-        issue_pv(0, j);
-        if (next) {
-          if (!mbar_wait(&k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
+        issue_s(0, gk);
+        if (has_b) issue_s(1, gk);
+        mma_commit(&k_empty[gk & 1]);
+        if (nt == 1) mma_commit(&q_empty);  // last S of this block issued
+        for (int j = 0; j < nt; ++j) {
+          const uint32_t g = gk + j;
+          const bool next = j + 1 < nt;
+          if (!mbar_wait(&v_full[g & 1], (g >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN) ||
+              !mbar_wait(&p_full[0], gp[0] & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
-          issue_s(0, j + 1);
+          issue_pv(0, g, j);
+          ++gp[0];
+          if (next) {
+            if (!mbar_wait(&k_full[(g + 1) & 1], ((g + 1) >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(0, g + 1);
+          }
+          if (has_b) {
+            if (!mbar_wait(&p_full[1], gp[1] & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_pv(1, g, j);
+            ++gp[1];
+          }
+          mma_commit(&v_empty[g & 1]);
+          if (next) {
+            if (has_b) issue_s(1, g + 1);
+            mma_commit(&k_empty[(g + 1) & 1]);
+            if (j + 2 == nt) mma_commit(&q_empty);  // last S of this block issued
+          }
         }
-        if (has_b) {
-          if (!mbar_wait(&p_full[1], j & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
-          tc_fence_after();
-          issue_pv(1, j);
-        }
-        mma_commit(&v_empty[j & 1]);
-        if (next) {
-          if (has_b) issue_s(1, j + 1);
-          mma_commit(&k_empty[(j + 1) & 1]);
-        }
+        gk += nt;
       }
       mma_commit(&done_bar);
       drain_wait(&done_bar, 0);
@@ -283,17 +325,21 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
   } else {
     // ---------------- softmax + output (warps 2..9) ----------------
     const int X = warp >= 6 ? 1 : 0;
-    if (X == 0 || has_b) {
-      const int quad = warp & 3;
-      const int r = quad * 32 + lane;  // query row in the tile == TMEM lane
-      const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
-      const uint32_t tS = tmem + lane_off + C::s_col(X);
-      const uint32_t tO = tmem + lane_off + C::o_col(X);
-      const float sl2 = 1.4426950408889634f / sqrtf((float)HD);  // log2(e) / sqrt(hd)
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;  // query row in the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + C::s_col(X);
+    const uint32_t tO = tmem + lane_off + C::o_col(X);
+    const float sl2 = 1.4426950408889634f / sqrtf((float)HD);  // log2(e) / sqrt(hd)
+    uint32_t gx = 0;  // tiles of this X processed so far (phases of s_full / p_full / pv_done)
+    bool ok = true;
+    for (int qb = qb0; qb < qb1 && ok; ++qb) {
+      const int q0 = qb * 2 * BQ;
+      if (X == 1 && !(q0 + BQ < p.Lq)) continue;  // this block has no tile B
+      const int qrow0 = c * p.Lq + q0;
       float m = -INFINITY, l = 0.0f;
-      bool ok = true;
-      for (int j = 0; j < nt; ++j) {
-        if (!warp_wait(&s_full[X], j & 1, &abort_flag, status)) { ok = false; break; }
+      for (int j = 0; j < nt; ++j, ++gx) {
+        if (!warp_wait(&s_full[X], gx & 1, &abort_flag, status)) { ok = false; break; }
         tc_fence_after();
         float s[128];
 #pragma unroll
@@ -339,8 +385,8 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
         }
         tmem_wait_st();
         if (resc && j > 0) {
-          // O must hold PV of every earlier tile before it is rescaled
-          if (!warp_wait(&pv_done[X], (j - 1) & 1, &abort_flag, status)) { ok = false; break; }
+          // O must hold PV of every earlier tile of this block before it is rescaled
+          if (!warp_wait(&pv_done[X], (gx - 1) & 1, &abort_flag, status)) { ok = false; break; }
           tc_fence_after();
           const float corr = ex2_approx(m - m_use);
           l *= corr;
@@ -354,36 +400,36 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
           }
         }
         {
-          float t0, t1, t2, t3;
+          float t0, t1;
           f2_unpack(f2_add(f2_add(sp2[0], sp2[1]), f2_add(sp2[2], sp2[3])), t0, t1);
-          (void)t2;
-          (void)t3;
           l += t0 + t1;
         }
         m = m_use;
         tc_fence_before();
         mbar_arrive(&p_full[X]);
       }
-      if (ok && nt > 0 && warp_wait(&pv_done[X], (nt - 1) & 1, &abort_flag, status)) {
-        tc_fence_after();
-        const float inv = 1.0f / l;
-        const bool row_ok = q0 + X * BQ + r < p.Lq;
-        bf16* O = (bf16*)p.out + (long long)(qrow0 + X * BQ + r) * p.ldo + h * HD;
+      if (!ok || nt == 0) break;
+      if (!warp_wait(&pv_done[X], (gx - 1) & 1, &abort_flag, status)) { ok = false; break; }
+      tc_fence_after();
+      const float inv = 1.0f / l;
+      const bool row_ok = q0 + X * BQ + r < p.Lq;
+      bf16* O = (bf16*)p.out + (long long)(qrow0 + X * BQ + r) * p.ldo + h * HD;
 #pragma unroll 1
-        for (int i = 0; i < HD / 32; ++i) {
-          float t[32];
-          tmem_ld32(tO + i * 32, t);
-          if (row_ok) {
-            uint4* d4 = reinterpret_cast<uint4*>(O + i * 32);
+      for (int i = 0; i < HD / 32; ++i) {
+        float t[32];
+        tmem_ld32(tO + i * 32, t);
+        if (row_ok) {
+          uint4* d4 = reinterpret_cast<uint4*>(O + i * 32);
 #pragma unroll
-            for (int q4 = 0; q4 < 4; ++q4)
-              d4[q4] = make_uint4(pack_bf16(t[q4 * 8] * inv, t[q4 * 8 + 1] * inv),
-                                  pack_bf16(t[q4 * 8 + 2] * inv, t[q4 * 8 + 3] * inv),
-                                  pack_bf16(t[q4 * 8 + 4] * inv, t[q4 * 8 + 5] * inv),
-                                  pack_bf16(t[q4 * 8 + 6] * inv, t[q4 * 8 + 7] * inv));
-          }
+          for (int q4 = 0; q4 < 4; ++q4)
+            d4[q4] = make_uint4(pack_bf16(t[q4 * 8] * inv, t[q4 * 8 + 1] * inv),
+                                pack_bf16(t[q4 * 8 + 2] * inv, t[q4 * 8 + 3] * inv),
+                                pack_bf16(t[q4 * 8 + 4] * inv, t[q4 * 8 + 5] * inv),
+                                pack_bf16(t[q4 * 8 + 6] * inv, t[q4 * 8 + 7] * inv));
         }
       }
+      // the next block's PV overwrites O only after this thread's next P arrives
+      tc_fence_before();
     }
   }
   tc_fence_before();
@@ -417,9 +463,15 @@ cudaError_t launch(const AttnParams& p, int* status, cudaStream_t s) {
     maps.kp = maps.k;
     maps.vp = maps.v;
   }
-  dim3 grid((p.Lq + 2 * BQ - 1) / (2 * BQ), p.n_heads, p.n_chunks);
+  // query blocks of 256 per CTA: more when the key set is short (the setup of
+  // a CTA, its Q loads and its O write-back are then amortised over more work)
+  const long long keys = (long long)p.Lk * (1 + (p.pred_in_batch ? 1 : 0) + (p.succ_in_batch ? 1 : 0));
+  AttnParams q = p;
+  q.qblocks_per_cta = p.qblocks_per_cta > 0 ? p.qblocks_per_cta : (keys <= 1024 ? 4 : 1);
+  const int nqb = (p.Lq + 2 * BQ - 1) / (2 * BQ);
+  dim3 grid((nqb + q.qblocks_per_cta - 1) / q.qblocks_per_cta, p.n_heads, p.n_chunks);
   if (!status) status = op_status_word();
-  attn_tc_kernel<HD><<<grid, 320, C::SMEM, s>>>(maps, p, status);
+  attn_tc_kernel<HD><<<grid, 320, C::SMEM, s>>>(maps, q, status);
   return cudaGetLastError();
 }
 
