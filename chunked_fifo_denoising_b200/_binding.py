@@ -115,6 +115,7 @@ _SIGS = {
     "dp_op_attention": (C.c_int, [C.POINTER(dp_attn_args), C.c_void_p]),
     "dp_op_layernorm_mod": (C.c_int, [C.POINTER(dp_ln_args), C.c_void_p]),
     "dp_op_check": (C.c_int, [C.c_void_p]),
+    "dp_op_selftest_timeout": (C.c_int, [C.c_void_p]),
 }
 
 EXPORTED = sorted(_SIGS)
@@ -180,3 +181,4 @@ def dp_op_gemm(args, stream): return _call("dp_op_gemm", C.byref(args), stream)
 def dp_op_attention(args, stream): return _call("dp_op_attention", C.byref(args), stream)
 def dp_op_layernorm_mod(args, stream): return _call("dp_op_layernorm_mod", C.byref(args), stream)
 def dp_op_check(stream): return _call("dp_op_check", stream)
+def dp_op_selftest_timeout(stream): return _call("dp_op_selftest_timeout", stream)

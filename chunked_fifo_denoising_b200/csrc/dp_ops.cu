@@ -110,6 +110,13 @@ dp_status dp_op_attention(const dp_attn_args* a, void* stream) {
   return DP_OK;
 }
 
+dp_status dp_op_selftest_timeout(void* stream) {
+  clear_error();
+  cudaError_t err = selftest_timeout(static_cast<cudaStream_t>(stream));
+  if (err != cudaSuccess) return fail(DP_ERR_CUDA, "self test launch: %s", cudaGetErrorString(err));
+  return DP_OK;
+}
+
 dp_status dp_op_check(void* stream) {
   clear_error();
   DP_CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));

@@ -443,12 +443,17 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
 template <int HD>
 cudaError_t launch(const AttnParams& p, int* status, cudaStream_t s) {
   using C = Cfg<HD>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(attn_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-  });
-  if (attr_err != cudaSuccess) return attr_err;
+  // the shared-memory opt-in is a per-device attribute of the function
+  static bool done[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!done[dev]) {
+    err = cudaFuncSetAttribute(attn_tc_kernel<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (err != cudaSuccess) return err;
+    done[dev] = true;
+  }
   const int w = p.n_heads * HD;
   AttnMaps maps;
   const long long q_rows = (long long)p.n_chunks * p.Lq;
@@ -476,6 +481,28 @@ cudaError_t launch(const AttnParams& p, int* status, cudaStream_t s) {
 }
 
 }  // namespace
+
+// One bounded wait on an mbarrier that nothing arrives at: exercises the
+// give-up path of the tensor-core kernels (status word set, clean exit).
+__global__ void selftest_timeout_kernel(int* status) {
+  __shared__ uint64_t bar;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, status, ST_TIMEOUT_ATTN);
+  __syncthreads();
+}
+
+cudaError_t selftest_timeout(cudaStream_t s) {
+  int* status = op_status_word();
+  if (!status) return cudaErrorInvalidValue;
+  selftest_timeout_kernel<<<1, 32, 0, s>>>(status);
+  return cudaGetLastError();
+}
 
 bool attention_tc_supported(const AttnParams& p) {
   if (p.f32 || (p.head_dim != 64 && p.head_dim != 128)) return false;

@@ -463,13 +463,17 @@ template <int BN, int STAGES>
 static cudaError_t launch_tc(const bf16* A, long long lda, const bf16* W, int M, int N, int K,
                              const EpiParams& e, int* status, cudaStream_t s) {
   constexpr int SMEM = STAGES * (BM * BK * 2 + BN * BK * 2) + 8 * 4096 + 1024;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>,
-                                    cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-  });
-  if (attr_err != cudaSuccess) return attr_err;
+  // the shared-memory opt-in is a per-device attribute of the function
+  static bool done[64] = {};
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!done[dev]) {
+    err = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    if (err != cudaSuccess) return err;
+    done[dev] = true;
+  }
   GemmMaps maps;
   memset(&maps, 0, sizeof(maps));
   if (!make_tmap(&maps.a, false, A, M, K, lda, BM, BK)) return cudaErrorInvalidValue;

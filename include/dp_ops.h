@@ -102,6 +102,12 @@ typedef struct {
 } dp_ln_args;
 DP_API dp_status dp_op_layernorm_mod(const dp_ln_args* a, void* stream);
 
+/* Exercises the bounded-wait failure path: launches one block that waits on
+ * an mbarrier nothing arrives at, gives up after the kernels' wait limit
+ * (2 s), sets the status word and returns; nothing faults.  A following
+ * dp_op_check must then report DP_ERR_KERNEL (and clear the word). */
+DP_API dp_status dp_op_selftest_timeout(void* stream);
+
 /* Waits for `stream`, then reads and clears the status word that the
  * tensor-core kernels of the calls above set when one of their bounded waits
  * gives up (they then skip the rest of their work).  DP_ERR_KERNEL if set. */

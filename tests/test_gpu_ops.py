@@ -292,3 +292,16 @@ def test_layernorm_mod(out_dtype, M, d):
     t = f64(table)[f64(sel).astype(int)[np.minimum(np.arange(M) // rpc, 3)]]
     ref = dit.modulate(dit.layer_norm(f64(x)), t[:, :d], t[:, d:])
     assert rel_l2(f64(out), ref) < (5e-3 if out_dtype == "bf16" else 1e-6)
+
+
+def test_bounded_wait_gives_up_and_reports():
+    """A kernel whose mbarrier is never completed gives up after the wait limit,
+    sets the status word (reported once as DP_ERR_KERNEL) and leaves the
+    context usable: the next GEMM runs and checks clean."""
+    s = torch.cuda.current_stream().cuda_stream
+    assert B.dp_op_check(s) == 0
+    assert B.dp_op_selftest_timeout(s) == 0
+    assert B.dp_op_check(s) == B.DP_ERR_KERNEL
+    assert "bounded wait" in B.dp_last_error()
+    assert B.dp_op_check(s) == 0          # the word was cleared
+    test_gemm_store_bf16(300, 256, 128)   # and kernels still run
