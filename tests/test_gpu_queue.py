@@ -86,6 +86,71 @@ def test_tiny_fp32_stream_matches_oracle(neighbours, rope):
     model.close()
 
 
+@pytest.mark.parametrize("precision,T,N", [("fp32", 1, 3), ("fp32", 4, 1), ("fp32", 6, 3),
+                                             ("bf16", 1, 3)])
+def test_degenerate_queues_match_oracle(precision, T, N):
+    """T = 1 (every step persists the head's K/V and each chunk's neighbour comes
+    from the cache), a single chunk, and a stream shorter than the queue, on
+    the tiny model (fp32: 1e-4 on every popped chunk; bf16: 2e-2)."""
+    w = synth.WORKLOADS["tiny_fp32"]
+    if precision == "bf16":  # bf16 path needs head_dim 64: 64 wide, one head
+        import dataclasses
+        w = dataclasses.replace(w, model=dataclasses.replace(w.model, n_heads=1))
+    m, q = w.model, w.queue
+    model, queue, p, text = make(w, precision, n_chunks=N, T=T)
+    noise = [synth.make_noise(m, q, k) for k in range(N)]
+    fn = dit.make_velocity_fn(p, text, m, T)
+    ready, traces = fifo.run_stream(fn, lambda k: noise[k], T, N)
+    assert len(traces) == N + T - 1
+    out = np.empty(q.chunk_shape(m), np.float32)
+    got = {}
+    for tr in traces:
+        queue.step(noise[tr.step] if tr.step < N else None)
+        while True:
+            st, cid = queue.try_pop(out)
+            if st != 0:
+                break
+            got[cid] = out.copy()
+    queue.sync()
+    assert sorted(got) == list(range(N))
+    tol = 1e-4 if precision == "fp32" else 2e-2
+    for k, ref in ready:
+        assert rel_l2(got[k], ref) <= tol, (k, rel_l2(got[k], ref))
+    model.close()
+
+
+def test_invalid_configurations_are_rejected():
+    import ctypes as C
+    from chunked_fifo_denoising_b200 import Model, Queue, DPError
+    from chunked_fifo_denoising_b200 import _binding as B
+    w = synth.WORKLOADS["tiny_fp32"]
+    m, q = w.model, w.queue
+    import dataclasses
+    with pytest.raises(DPError) as e:   # bf16 needs head_dim 64 or 128 (here 16)
+        Model(m, "bf16")
+    assert e.value.status == B.DP_ERR_INVALID_ARG
+    with pytest.raises(DPError):
+        Model(dataclasses.replace(m, n_heads=3), "fp32")
+    model = Model(m, "fp32")
+    text = synth.make_text(m)
+    with pytest.raises(DPError) as e:   # parameters not set yet
+        Queue(model, text, q.T, q.frames_per_chunk, q.lat_h, q.lat_w, 4)
+    assert e.value.status == B.DP_ERR_STATE
+    model.set_params(synth.make_params(m))
+    for kw in (dict(T=0), dict(n=0), dict(lat_h=7)):
+        with pytest.raises(DPError) as e:
+            Queue(model, text, kw.get("T", q.T), q.frames_per_chunk, kw.get("lat_h", q.lat_h), q.lat_w,
+                  kw.get("n", 4))
+        assert e.value.status == B.DP_ERR_INVALID_ARG
+    with pytest.raises(DPError):        # wrong element count
+        model.set_param("patch.w", np.zeros(5, np.float32))
+    queue = Queue(model, text, q.T, q.frames_per_chunk, q.lat_h, q.lat_w, 4)
+    with pytest.raises(DPError):        # read_latents with a wrong count
+        queue.read_latents(3)
+    assert B.dp_queue_step(None, None, 0) == B.DP_ERR_INVALID_ARG
+    model.close()
+
+
 @pytest.mark.parametrize("name", list(synth.WORKLOADS))
 def test_bookkeeping_exact_on_every_schedule(name):
     """The (T, N) schedule of each workload, run at full N on the tiny model."""
