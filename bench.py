@@ -257,6 +257,8 @@ def run_ours(args, w):
     # random-init weights on the device, N(0, 0.02^2), seeded per rank
     g = torch.Generator(device="cuda").manual_seed(1000 + rank)
     import synth
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
     model = Model(m, "bf16", stream=stream, neighbours=args.neighbours)
     for name, shape, per_layer in synth.param_specs(m):
         for l in range(m.n_layers if per_layer else 1):
@@ -266,17 +268,30 @@ def run_ours(args, w):
             model.set_param(name, t, l)
             del t
     text = torch.randn((m.text_len, m.text_in_dim), generator=g, device="cuda")
-    n_chunks = T - 1 + args.warmup + args.steps + args.e2e_steps + 2
+    n_chunks = T + 1 + args.warmup + args.steps + args.e2e_steps + 2
+    torch.cuda.synchronize()
+    free1 = torch.cuda.mem_get_info()[0]
     queue = Queue(model, text, T, q.frames_per_chunk, q.lat_h, q.lat_w, n_chunks,
                   ready_capacity=2, seed=3 + rank)
+    torch.cuda.synchronize()
+    free2 = torch.cuda.mem_get_info()[0]
     out = torch.empty(queue.chunk_shape, device="cuda")
-    # fill: T-1 steps bring the queue to full occupancy (untimed)
-    for _ in range(T - 1):
-        queue.step(None)
-        queue.try_pop(out)
+    if args.fill == "steps":
+        # T-1 real steps bring the queue to full occupancy (untimed)
+        for _ in range(T - 1):
+            queue.step(None)
+            queue.try_pop(out)
+    else:
+        # the steady state placed directly: chunks 1..T at levels 1..T, and the
+        # persisted K/V of chunk 0 (popped last step) for the head's predecessor
+        lat = torch.randn((T,) + queue.chunk_shape, generator=g, device="cuda")
+        kv = torch.randn((m.n_layers, 2, queue.tokens, m.dim), generator=g, device="cuda")
+        queue.load_state(T, T + 1, lat, kv)
+        del lat, kv
     queue.sync()
     info = queue.inspect()
     assert info["n"] == occ, info
+    assert info["head_pred"] != 0, info
     for _ in range(args.warmup):
         queue.step(None)
         queue.pop(out)
@@ -356,7 +371,10 @@ def run_ours(args, w):
                         for k, v in kt.items() if v["launches"]},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(hn.numel() * 4),
                     "d2h_bytes_per_step": int(ho.numel() * 4), "steps": args.e2e_steps},
-            "gpu_launches": launches, "clocks": ck}
+            "gpu_launches": launches, "clocks": ck,
+            "memory": {"model_bytes": int(free0 - free1), "queue_bytes": int(free1 - free2),
+                       "source": "cudaMemGetInfo around dp_model_create+set_param and dp_queue_init"},
+            "fill": args.fill}
     if attn["ms"] > 0:
         line["self_attention_tflops"] = attn["flops"] / (attn["ms"] / 1e3) / 1e12
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -381,6 +399,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="wan1.3b_480p")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fill", default="steps", choices=["steps", "load"],
+                    help="reach the steady state by T-1 real steps, or place it with "
+                         "dp_queue_load_state (random latents and persisted K/V)")
     ap.add_argument("--qk-norm-rope", action="store_true",
                     help="per-head QK RMSNorm and 3-D rotary positions in self-attention")
     ap.add_argument("--neighbours", default="pred", choices=["pred", "both"],

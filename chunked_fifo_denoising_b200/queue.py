@@ -168,10 +168,17 @@ class Queue:
         return out
 
     def load_state(self, step, n_pushed, latents, pred_kv=None):
-        lat = np.ascontiguousarray(latents, np.float32)
-        kv = None if pred_kv is None else np.ascontiguousarray(pred_kv, np.float32)
-        B.check(B.dp_queue_load_state(self.handle, step, n_pushed, lat.shape[0], lat.ctypes.data,
-                                      None if kv is None else kv.ctypes.data, B.DP_LOC_HOST),
+        """latents [n][C][F][H][W] and pred_kv [layers][2][tokens][dim], float32:
+        numpy arrays (host) or torch tensors, both at the same location."""
+        if isinstance(latents, np.ndarray) or not hasattr(latents, "data_ptr"):
+            latents = np.ascontiguousarray(latents, np.float32)
+            if pred_kv is not None:
+                pred_kv = np.ascontiguousarray(pred_kv, np.float32)
+        lat, loc = _ptr(latents)
+        kv, kv_loc = _ptr(pred_kv)
+        if pred_kv is not None and kv_loc != loc:
+            raise ValueError("latents and pred_kv must be at the same location")
+        B.check(B.dp_queue_load_state(self.handle, step, n_pushed, latents.shape[0], lat, kv, loc),
                 "dp_queue_load_state")
 
     def read_pred_kv(self):

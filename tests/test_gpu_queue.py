@@ -368,10 +368,11 @@ def test_coordinated_noise_pushes_the_oracle_frames():
 
 
 def test_device_memory_flat_in_stream_length():
-    """Long-stream workload: memory after init is the same for 32, 64 and 128
-    chunks and the steps allocate nothing (two-layer model, zero weights)."""
+    """Long-stream workload (Wan-1.3B shapes, all 30 layers, zero weights):
+    device memory after init is the same for 32, 64 and 128 chunks and the
+    steps allocate nothing."""
     from chunked_fifo_denoising_b200 import Model, Queue
-    w = synth.truncated(synth.WORKLOADS["wan1.3b_480p_long"], 2)
+    w = synth.WORKLOADS["wan1.3b_480p_long"]
     m, q = w.model, w.queue
     model = Model(m, "bf16")
     for name, shape, per_layer in synth.param_specs(m):
@@ -391,5 +392,6 @@ def test_device_memory_flat_in_stream_length():
         assert free2 == free1
         used.append(free0 - free1)
         queue.close()
+    print(f"queue device bytes at N = 32, 64, 128: {used}")
     assert used[0] == used[1] == used[2]
     model.close()
