@@ -282,11 +282,12 @@ def run_ours(args, w):
             queue.step(None)
             queue.try_pop(out)
     else:
-        # the steady state placed directly: chunks 1..T at levels 1..T, and the
-        # persisted K/V of chunk 0 (popped last step) for the head's predecessor
-        lat = torch.randn((T,) + queue.chunk_shape, generator=g, device="cuda")
+        # the steady state placed directly: chunks 1..T-1 at levels 1..T-1 (the
+        # step pushes chunk T at level T), and the persisted K/V of chunk 0
+        # (popped last step) for the head's predecessor
+        lat = torch.randn((T - 1,) + queue.chunk_shape, generator=g, device="cuda")
         kv = torch.randn((m.n_layers, 2, queue.tokens, m.dim), generator=g, device="cuda")
-        queue.load_state(T, T + 1, lat, kv)
+        queue.load_state(T, T, lat, kv)
         del lat, kv
     queue.sync()
     info = queue.inspect()

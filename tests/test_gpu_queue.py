@@ -379,6 +379,13 @@ def test_device_memory_flat_in_stream_length():
         t = torch.zeros(shape, device="cuda")
         model.set_params({name: [t] * m.n_layers if per_layer else t})
     text = torch.zeros((m.text_len, m.text_in_dim), device="cuda")
+    # the driver loads each kernel's module at its first launch: load them all
+    # with a throwaway queue before measuring
+    warm = Queue(model, text, q.T, q.frames_per_chunk, q.lat_h, q.lat_w, 4)
+    for _ in range(3):
+        warm.step(None)
+    warm.sync()
+    warm.close()
     torch.cuda.synchronize()
     used = []
     for n in (32, 64, 128):
@@ -389,6 +396,7 @@ def test_device_memory_flat_in_stream_length():
             queue.step(None)
         queue.sync()
         free2 = torch.cuda.mem_get_info()[0]
+        print(f"N = {n}: queue device bytes {free0 - free1}, allocated by 3 steps {free1 - free2}")
         assert free2 == free1
         used.append(free0 - free1)
         queue.close()
