@@ -197,6 +197,51 @@ def max_over_ranks(values, dist=None, device=None):
     return [float(x) for x in t]
 
 
+def measure_plateau(model, m, q, text, occ, steps, warmup, g, dist, world, rank, peak_tf):
+    """A stream shorter than the queue never fills it: from the push of its
+    last chunk until its first chunk pops, `occ` chunks advance one level per
+    step with no push and no pop.  Places that state (chunks 0 .. occ-1 at
+    levels T-occ .. T-1, chunk 0 without a predecessor) and times `steps`
+    plateau steps.  A chunk needs T steps, so the stream's rate is
+    occ / T chunks per step."""
+    import torch
+
+    from chunked_fifo_denoising_b200 import Queue
+    T = q.T
+    if warmup + steps > T - occ:
+        raise SystemExit(f"plateau of {T - occ} steps is shorter than warm-up + steps")
+    queue = Queue(model, text, T, q.frames_per_chunk, q.lat_h, q.lat_w, occ, ready_capacity=2,
+                  seed=3 + rank)
+    lat = torch.randn((occ,) + queue.chunk_shape, generator=g, device="cuda")
+    queue.load_state(occ, occ, lat)
+    del lat
+    info = queue.inspect()
+    assert info["n"] == occ and info["head_pred"] == 0 and info["levels"][0] == T - occ, info
+    for _ in range(warmup):
+        queue.step(None)
+    queue.sync()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        queue.step(None)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks([e0.elapsed_time(e1)], dist, device="cuda")[0]
+    queue.sync()
+    queue.close()
+    Lc = q.tokens_per_chunk(m)
+    flops = step_flops(m, q, occ) - m.n_layers * 4.0 * Lc * Lc * m.dim  # chunk 0: own keys only
+    step_s = ms / steps / 1e3
+    return {"occupancy": occ, "steps": steps, "warmup": warmup, "ms_per_step": ms / steps,
+            "value": world * occ * q.frames_per_chunk / T / step_s, "unit": UNIT,
+            "step_tflop": flops / 1e12, "pct_bf16_peak": 100.0 * flops / step_s / (peak_tf * 1e12)}
+
+
 def whole_job_rate(world, steps, frames_per_step, ms):
     """Units of all ranks (weak scaling: each rank runs its own replica) over
     the slowest rank's time."""
@@ -378,6 +423,13 @@ def run_ours(args, w):
             "fill": args.fill}
     if attn["ms"] > 0:
         line["self_attention_tflops"] = attn["flops"] / (attn["ms"] / 1e3) / 1e12
+    if args.plateau:
+        if 0 < q.n_chunks < T:
+            queue.close()
+            line["plateau"] = measure_plateau(model, m, q, text, q.n_chunks, args.steps, args.warmup, g,
+                                              dist, world, rank, peak_tf)
+        else:
+            line["plateau"] = None  # the stream fills the queue: its steady state is the full step
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, t, threads = oracle_sample(w)
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
@@ -400,6 +452,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="wan1.3b_480p")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--plateau", action="store_true",
+                    help="also time the plateau of the workload's own stream length when it is "
+                         "shorter than the queue (no push, no pop; rate = occupancy / T chunks per step)")
     ap.add_argument("--fill", default="steps", choices=["steps", "load"],
                     help="reach the steady state by T-1 real steps, or place it with "
                          "dp_queue_load_state (random latents and persisted K/V)")
