@@ -337,7 +337,9 @@ def run_ours(args, w):
     queue.sync()
     info = queue.inspect()
     assert info["n"] == occ, info
-    assert info["head_pred"] != 0, info
+    # placed state: the head reads its predecessor's persisted K/V (after a real
+    # fill the first warm-up step's head is chunk 0, which has none)
+    assert args.fill == "steps" or info["head_pred"] != 0, info
     for _ in range(args.warmup):
         queue.step(None)
         queue.pop(out)

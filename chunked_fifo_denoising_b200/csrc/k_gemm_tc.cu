@@ -15,6 +15,15 @@
 //               overlap this tile's epilogue.
 // Tiles are walked row-block-major so the CTAs in flight share A row blocks
 // through L2 while W stays L2-resident.  Every mbarrier wait is bounded.
+//
+// Pair mode (PAIR, N a multiple of 256): clusters of two CTAs on two SMs
+// compute 256 x 256 tiles with tcgen05.mma.cta_group::2 (M = 256).  Each CTA
+// loads its own 128 rows of A and 128 of the 256 rows of W, so an SM streams
+// 64 instead of 96 bytes of operands per 8192 MMA FLOP.  The first CTA of the
+// pair waits for both CTAs' loads on its own full barriers, issues the MMAs
+// and commits them to the empty and accumulator barriers of both CTAs; each
+// CTA runs the epilogue of its own 128 rows from its own tensor memory and
+// releases the accumulator to the first CTA.  No load is multicast.
 #include <cstring>
 #include <mutex>
 
@@ -27,20 +36,6 @@ using namespace tc;
 namespace {
 
 constexpr int BM = 128, BK = 64;
-
-__device__ __forceinline__ void store_bf16x32(bf16* dst, const float (&v)[32]) {
-  uint4* d4 = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint32_t w[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      __nv_bfloat162 p = __floats2bfloat162_rn(v[8 * i + 2 * j], v[8 * i + 2 * j + 1]);
-      w[j] = *reinterpret_cast<uint32_t*>(&p);
-    }
-    d4[i] = make_uint4(w[0], w[1], w[2], w[3]);
-  }
-}
 
 // Bias (and activation) for `n` consecutive columns starting at col0; columns
 // at or beyond N read no bias.
@@ -87,18 +82,20 @@ struct GemmMaps {
   CUtensorMap res;     // fp32 residual stream for the reduce-add epilogues
 };
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool PAIR>
 __global__ void __launch_bounds__(320, 1)
 gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiParams e, int* status) {
+  constexpr int BNL = PAIR ? BN / 2 : BN;  // rows of W this CTA loads per tile
+  constexpr int TM = PAIR ? 2 * BM : BM;   // rows of an output tile
   constexpr uint32_t A_BYTES = BM * BK * 2;
-  constexpr uint32_t B_BYTES = BN * BK * 2;
+  constexpr uint32_t B_BYTES = BNL * BK * 2;
   constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;
   constexpr uint32_t STG_OFF = STAGES * STAGE_BYTES;  // 8 warps x one 4 KB staging box
   // columns per epilogue warp; with BN = 64 the second warp group has no columns
   // and only keeps in step with the accumulator barriers
   constexpr int HALF = BN >= 128 ? BN / 2 : BN;
   constexpr uint32_t TMEM_COLS = 2 * BN;
-  constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, 0, 0);
+  constexpr uint32_t IDESC = idesc_bf16_f32(TM, BN, 0, 0);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -107,8 +104,14 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
   __shared__ volatile int abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // pair mode: CTA `rank` of the pair owns rows rank*128.. of every tile; the
+  // pairs walk the tiles together
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int unit0 = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  const int units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   const int tiles_n = (N + BN - 1) / BN;
-  const int tiles_m = (M + BM - 1) / BM;
+  const int tiles_m = (M + TM - 1) / TM;
   const int num_tiles = tiles_n * tiles_m;
   const int kblocks = K / BK;
 
@@ -119,15 +122,20 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&tfull_bar[i], 1);
-      mbar_init(&tempty_bar[i], 256);
+      mbar_init(&tempty_bar[i], PAIR ? 16 : 256);  // pair: one arrival per epilogue warp of each CTA
     }
     mbar_init(&done_bar, 1);
     abort_flag = 0;
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(&tmem_base_sh, TMEM_COLS);
-    tmem_relinquish();
+    if (PAIR) {
+      tmem_alloc_pair(&tmem_base_sh, TMEM_COLS);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(&tmem_base_sh, TMEM_COLS);
+      tmem_relinquish();
+    }
   }
   if (warp == 0 && lane == 0) {
     prefetch_tmap(&maps.a);
@@ -135,6 +143,7 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
   }
   tc_fence_before();
   __syncthreads();
+  if (PAIR) cluster_sync();  // the peer's barriers are initialised before any remote signal
   tc_fence_after();
   const uint32_t tmem_base = tmem_base_sh;
 
@@ -145,17 +154,25 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
       uint32_t phase = 0;
       uint32_t issued = 0, issued_par = 0;  // per-stage bit masks for the drain
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
+      for (int t = unit0; t < num_tiles && ok; t += units) {
+        const int m0 = (t / tiles_n) * TM + (int)rank * BM, n0 = (t % tiles_n) * BN + (int)rank * BNL;
         for (int kb = 0; kb < kblocks; ++kb) {
           if (!mbar_wait(&empty_bar[stage], phase ^ 1, &abort_flag, status, ST_TIMEOUT_GEMM)) {
             ok = false;
             break;
           }
           uint8_t* sa = smem + stage * STAGE_BYTES;
-          mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
-          tma_load_2d(sa, &maps.a, kb * BK, m0, &full_bar[stage]);
-          tma_load_2d(sa + A_BYTES, &maps.b, kb * BK, n0, &full_bar[stage]);
+          if (PAIR) {
+            // both CTAs' bytes land on the first CTA's full barrier
+            if (leader) mbar_arrive_expect_tx(&full_bar[stage], 2 * STAGE_BYTES);
+            const uint32_t fb = cluster_addr(&full_bar[stage], 0);
+            tma_load_2d_pair(sa, &maps.a, kb * BK, m0, fb);
+            tma_load_2d_pair(sa + A_BYTES, &maps.b, kb * BK, n0, fb);
+          } else {
+            mbar_arrive_expect_tx(&full_bar[stage], STAGE_BYTES);
+            tma_load_2d(sa, &maps.a, kb * BK, m0, &full_bar[stage]);
+            tma_load_2d(sa + A_BYTES, &maps.b, kb * BK, n0, &full_bar[stage]);
+          }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -164,19 +181,26 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
           }
         }
       }
-      if (abort_flag) {  // let copies in flight land before the CTA exits
+      // the second CTA of a pair cannot see its copies complete (they count on
+      // the first CTA's barriers): after a give-up it lets them settle for 1 ms
+      if (abort_flag && !leader && issued) {
+        const unsigned long long t0 = globaltimer();
+        while (globaltimer() - t0 < 1000000ull) {
+        }
+      }
+      if (abort_flag && leader) {  // let copies in flight land before the CTA exits
         for (int s = 0; s < STAGES; ++s)
           if (issued & (1u << s)) drain_wait(&full_bar[s], (issued_par >> s) & 1u);
       }
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ---------------- MMA issuer ----------------
+    if (lane == 0 && leader) {
+      // ---------------- MMA issuer (the first CTA of a pair) ----------------
       int stage = 0;
       uint32_t phase = 0;
       int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++it) {
+      for (int t = unit0; t < num_tiles && ok; t += units, ++it) {
         const int buf = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
         if (!mbar_wait(&tempty_bar[buf], acc_phase ^ 1, &abort_flag, status, ST_TIMEOUT_GEMM)) break;
@@ -192,17 +216,30 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
           const uint64_t ad = desc_sw128(sa, 16, 1024);
           const uint64_t bd = desc_sw128(sa + A_BYTES, 16, 1024);
 #pragma unroll
-          for (int k = 0; k < BK / 16; ++k)  // +32 bytes along K per step = +2 in the address field
-            mma_bf16_ss(dtm, ad + 2 * k, bd + 2 * k, IDESC, (kb | k) != 0);
-          mma_commit(&empty_bar[stage]);
+          for (int k = 0; k < BK / 16; ++k) {  // +32 bytes along K per step = +2 in the address field
+            if (PAIR) mma_bf16_ss_pair(dtm, ad + 2 * k, bd + 2 * k, IDESC, (kb | k) != 0);
+            else mma_bf16_ss(dtm, ad + 2 * k, bd + 2 * k, IDESC, (kb | k) != 0);
+          }
+          if (PAIR) {
+            mma_commit_pair_both(&empty_bar[stage]);
+          } else {
+            mma_commit(&empty_bar[stage]);
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
           }
         }
-        if (ok) mma_commit(&tfull_bar[buf]);
+        if (ok) {
+          if (PAIR) {
+            mma_commit_pair_both(&tfull_bar[buf]);
+          } else {
+            mma_commit(&tfull_bar[buf]);
+          }
+        }
       }
-      mma_commit(&done_bar);
+      if (PAIR) mma_commit_pair(&done_bar);
+      else mma_commit(&done_bar);
       drain_wait(&done_bar, 0);
     }
     __syncwarp();
@@ -215,14 +252,14 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
     const bool bf16_out = (e.mode == EPI_STORE && !e.out_f32) || e.mode == EPI_GELU;
     const bool reduce = e.mode == EPI_RESID || e.mode == EPI_RESID_GATED;
     int it = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+    for (int t = unit0; t < num_tiles; t += units, ++it) {
       const int buf = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       // warp-uniform: the TMEM loads below are warp-collective
       const bool waited = mbar_wait(&tfull_bar[buf], acc_phase, &abort_flag, status, ST_TIMEOUT_GEMM);
       if (!__all_sync(0xffffffffu, waited)) break;
       tc_fence_after();
-      const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN + half * HALF;
+      const int m0 = (t / tiles_n) * TM + (int)rank * BM, n0 = (t % tiles_n) * BN + half * HALF;
       const int row_base = m0 + quad * 32;
       const int row = row_base + lane;
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + half * HALF;
@@ -385,16 +422,26 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
         }
       }
       tc_fence_before();
-      mbar_arrive(&tempty_bar[buf]);
+      if (PAIR) {
+        __syncwarp();  // every lane's accumulator loads are complete
+        if (lane == 0) mbar_arrive_cluster(cluster_addr(&tempty_bar[buf], 0));
+      } else {
+        mbar_arrive(&tempty_bar[buf]);
+      }
     }
     if (lane == 0) bulk_wait_all();  // stores and reductions have landed
   }
   tc_fence_before();
   __syncthreads();
+  // pair: neither CTA frees tensor memory or leaves while the other may still
+  // signal its barriers or the MMAs may still read its shared memory
+  if (PAIR) cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else tmem_dealloc(tmem_base, TMEM_COLS);
   }
+  if (PAIR) cluster_sync();
 }
 
 // ---------------------------------------------------------------------------
@@ -459,10 +506,12 @@ bool gemm_tc_supported(long long lda, int M, int N, int K) {
   return M > 0 && N > 0 && K > 0 && K % BK == 0 && N % 32 == 0 && lda % 8 == 0 && lda >= K;
 }
 
-template <int BN, int STAGES>
+template <int BN, int STAGES, bool PAIR>
 static cudaError_t launch_tc(const bf16* A, long long lda, const bf16* W, int M, int N, int K,
                              const EpiParams& e, int* status, cudaStream_t s) {
-  constexpr int SMEM = STAGES * (BM * BK * 2 + BN * BK * 2) + 8 * 4096 + 1024;
+  constexpr int BNL = PAIR ? BN / 2 : BN;
+  constexpr int TM = PAIR ? 2 * BM : BM;
+  constexpr int SMEM = STAGES * (BM * BK * 2 + BNL * BK * 2) + 8 * 4096 + 1024;
   // the shared-memory opt-in is a per-device attribute of the function
   static bool done[64] = {};
   int dev = 0;
@@ -470,14 +519,15 @@ static cudaError_t launch_tc(const bf16* A, long long lda, const bf16* W, int M,
   if (err != cudaSuccess) return err;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (!done[dev]) {
-    err = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES>, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    err = cudaFuncSetAttribute(gemm_tc_kernel<BN, STAGES, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               SMEM);
     if (err != cudaSuccess) return err;
     done[dev] = true;
   }
   GemmMaps maps;
   memset(&maps, 0, sizeof(maps));
   if (!make_tmap(&maps.a, false, A, M, K, lda, BM, BK)) return cudaErrorInvalidValue;
-  if (!make_tmap(&maps.b, false, W, N, K, K, BN, BK)) return cudaErrorInvalidValue;
+  if (!make_tmap(&maps.b, false, W, N, K, K, BNL, BK)) return cudaErrorInvalidValue;
   if (e.mode == EPI_GELU || (e.mode == EPI_STORE && !e.out_f32)) {
     if (!make_tmap(&maps.out, false, e.out, M, N, e.ldo, 32, 64)) return cudaErrorInvalidValue;
   } else if (e.mode == EPI_STORE) {
@@ -487,20 +537,46 @@ static cudaError_t launch_tc(const bf16* A, long long lda, const bf16* W, int M,
   } else if (e.mode != EPI_EULER) {
     return cudaErrorInvalidValue;
   }
-  const int tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-  const int grid = tiles < sm_count() ? tiles : sm_count();
+  const int tiles = ((M + TM - 1) / TM) * ((N + BN - 1) / BN);
   if (!status) status = op_status_word();
-  gemm_tc_kernel<BN, STAGES><<<grid, 320, SMEM, s>>>(maps, M, N, K, e, status);
-  return cudaGetLastError();
+  if (!PAIR) {
+    const int grid = tiles < sm_count() ? tiles : sm_count();
+    gemm_tc_kernel<BN, STAGES, PAIR><<<grid, 320, SMEM, s>>>(maps, M, N, K, e, status);
+    return cudaGetLastError();
+  }
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(320, 1, 1);
+  cfg.dynamicSmemBytes = SMEM;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // pairs that fit on the device at once (one CTA per SM)
+  static int max_pairs[64] = {};
+  if (!max_pairs[dev]) {
+    cfg.gridDim = dim3(2 * (sm_count() / 2), 1, 1);
+    int n = 0;
+    err = cudaOccupancyMaxActiveClusters(&n, gemm_tc_kernel<BN, STAGES, PAIR>, &cfg);
+    if (err != cudaSuccess) return err;
+    if (n <= 0) return cudaErrorInvalidConfiguration;
+    max_pairs[dev] = n;
+  }
+  const int pairs = tiles < max_pairs[dev] ? tiles : max_pairs[dev];
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  return cudaLaunchKernelEx(&cfg, gemm_tc_kernel<BN, STAGES, PAIR>, maps, M, N, K, e, status);
 }
 
 cudaError_t gemm_tc(const bf16* A, long long lda, const bf16* W, int M, int N, int K,
                     const EpiParams& e, int* status, cudaStream_t s) {
   if (!gemm_tc_supported(lda, M, N, K)) return cudaErrorInvalidValue;
   if ((reinterpret_cast<uintptr_t>(A) | reinterpret_cast<uintptr_t>(W)) & 15) return cudaErrorInvalidValue;
-  if (N % 256 == 0) return launch_tc<256, 4>(A, lda, W, M, N, K, e, status, s);
-  if (N % 128 == 0) return launch_tc<128, 6>(A, lda, W, M, N, K, e, status, s);
-  return launch_tc<64, 8>(A, lda, W, M, N, K, e, status, s);
+  if (N % 256 == 0) return launch_tc<256, 6, true>(A, lda, W, M, N, K, e, status, s);
+  if (N % 128 == 0) return launch_tc<128, 6, false>(A, lda, W, M, N, K, e, status, s);
+  return launch_tc<64, 8, false>(A, lda, W, M, N, K, e, status, s);
 }
 
 }  // namespace dp
