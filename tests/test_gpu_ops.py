@@ -69,9 +69,12 @@ def run_gemm(A, W, bias, epi, out=None, resid=None, gate=None, sel=None, rpc=1, 
 
 
 @pytest.mark.parametrize("M,N,K", [(300, 256, 128), (129, 64, 64), (1000, 384, 192),
-                                   (300, 192, 128), (200, 96, 64),
+                                   (300, 192, 128), (200, 96, 64), (100, 256, 64),
                                    (2048, 1536, 512), (257, 4608, 1536)])
 def test_gemm_store_bf16(M, N, K):
+    """N a multiple of 256 runs in CTA pairs (256-row tiles): M = 100 leaves the
+    second CTA of the only pair without rows, M = 257 and 300 leave the second
+    CTA of the last pair without rows; N = 64, 96, 192, 384 take single CTAs."""
     A, W = gen((M, K), seed=1), gen((N, K), 0.02, seed=2)
     bias = gen((N,), 0.02, torch.float32, seed=3)
     out = torch.empty((M, N), device="cuda", dtype=torch.bfloat16)
