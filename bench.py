@@ -437,6 +437,14 @@ def run_ours(args, w):
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle",
                                 "sample": f"1 chunk x 1 layer of the step ({t:.1f} s), scaled by "
                                           f"T x layers = {T * m.n_layers}; float64 numpy"}
+        try:  # the same sample with the BLAS pool held to one thread
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                v1, t1, _ = oracle_sample(w)
+            line["cpu_baseline"]["one_thread"] = {"value": v1, "unit": UNIT, "cores": 1,
+                                                  "sample_s": round(t1, 2)}
+        except ImportError:
+            pass
     if rank == 0:
         print(json.dumps(line), flush=True)
     model.close()
