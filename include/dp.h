@@ -192,12 +192,19 @@ DP_API dp_status dp_queue_init(dp_model* m, const dp_queue_config* qc, const flo
  * DP_ERR_CUDA / DP_ERR_INVALID_ARG from a failed launch inside the step leave
  * part of the step enqueued: the queue must then be destroyed (or reloaded
  * with dp_queue_load_state).  A queue is not safe to use from several host
- * threads at once. */
+ * threads at once.
+ * Ownership: the step is asynchronous on the model's stream.  A device buffer,
+ * or a page-locked host buffer, is read when the stream reaches the push, so
+ * the caller must not overwrite it before the step completes (dp_queue_sync or
+ * a later event on the stream); a pageable host buffer is copied before the
+ * call returns. */
 DP_API dp_status dp_queue_step(dp_queue* q, const float* new_chunk_noise, dp_loc loc);
 
 /* Copies the oldest ready chunk ([C][F][H][W] fp32) to `out` at `loc` and
  * frees its slot; `chunk_id` (may be NULL) receives its id.  Chunk ids pop in
- * strictly increasing order.  DP_ERR_EMPTY if none is ready. */
+ * strictly increasing order.  DP_ERR_EMPTY if none is ready.  A host `out` is
+ * complete when the call returns (it waits for the stream); a device `out` is
+ * written in stream order. */
 DP_API dp_status dp_queue_pop(dp_queue* q, float* out, dp_loc loc, long long* chunk_id);
 
 /* Replaces the coordinated-noise pool (noise_mode 1) with `pool`
