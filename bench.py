@@ -10,10 +10,18 @@ frames/s (2 frames leave the queue per step) and the fraction of the bf16
 tensor-core peak reached by the step's algorithmic FLOPs.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--fill steps|load] [--plateau]
+                    [--neighbours pred|both] [--qk-norm-rope]
 
 N > 1 runs N independent replicas (one queue per GPU, no collective on the
 data path), launched by torch.distributed.run.  --impl reference times the
 float64 CPU oracle on a bounded sample of the same step (rank 0 only).
+--fill load places the steady state with dp_queue_load_state instead of T-1
+real steps (needed for the Wan-14B shapes, where a step takes seconds);
+--plateau also times the partial-queue steady state of a stream shorter than
+the queue.  Besides the metric, the line reports the roofline of the GEMM
+class, the per-class kernel times, end-to-end throughput with host buffers,
+clocks sampled during the timed region, device memory and the CPU oracle.
 """
 from __future__ import annotations
 
