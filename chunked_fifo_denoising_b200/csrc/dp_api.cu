@@ -732,6 +732,8 @@ static void free_queue(dp_queue* q) {
   if (q->h_slot) cudaFreeHost(q->h_slot);
   if (q->h_dsig) cudaFreeHost(q->h_dsig);
   if (q->table_ev) cudaEventDestroy(q->table_ev);
+  if (q->h_noise) cudaFreeHost(q->h_noise);
+  if (q->noise_ev) cudaEventDestroy(q->noise_ev);
   q->timer.release();
 }
 
@@ -878,6 +880,9 @@ dp_status dp_queue_init(dp_model* m, const dp_queue_config* qc, const float* tex
       e = cudaMallocHost(&q->h_rope_t, (size_t)qc->T * q->rope_Fq * q->rope_nt * 2 * sizeof(float));
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&q->table_ev, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventRecord(q->table_ev, m->stream);
+    if (e == cudaSuccess) e = cudaMallocHost(&q->h_noise, (size_t)q->chunk_numel * sizeof(float));
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&q->noise_ev, cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventRecord(q->noise_ev, m->stream);
     if (e != cudaSuccess) s = fail(DP_ERR_OOM, "pinned staging: %s", cudaGetErrorString(e));
   }
   if (s == DP_OK) s = build_tables(q, text, text_loc);
@@ -934,9 +939,15 @@ dp_status dp_queue_step(dp_queue* q, const float* noise, dp_loc loc) {
   cudaStream_t s = m->stream;
   if (pl.push) {
     float* slot = q->ring.as<float>() + (size_t)(q->next_id % q->n_slots) * q->chunk_numel;
-    if (noise) {
-      DP_CK(cudaMemcpyAsync(slot, noise, (size_t)q->chunk_numel * 4,
-                            loc == DP_LOC_HOST ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice, s));
+    if (noise && loc == DP_LOC_HOST) {
+      // the caller may reuse its host buffer once the call returns: stage it
+      // in pinned memory (the previous push has left the staging by now)
+      DP_CK(cudaEventSynchronize(q->noise_ev));
+      std::memcpy(q->h_noise, noise, (size_t)q->chunk_numel * 4);
+      DP_CK(cudaMemcpyAsync(slot, q->h_noise, (size_t)q->chunk_numel * 4, cudaMemcpyHostToDevice, s));
+      DP_CK(cudaEventRecord(q->noise_ev, s));
+    } else if (noise) {
+      DP_CK(cudaMemcpyAsync(slot, noise, (size_t)q->chunk_numel * 4, cudaMemcpyDeviceToDevice, s));
     } else if (q->qc.noise_mode == 1) {
       const int F = q->qc.frames_per_chunk;
       DP_CK(noise_from_pool(q->noise_pool.as<float>(), m->cfg.latent_ch, F,

@@ -101,6 +101,8 @@ struct dp_queue {
   int* h_slot = nullptr;
   float* h_dsig = nullptr;
   cudaEvent_t table_ev = nullptr;
+  float* h_noise = nullptr;           // pinned copy of a pushed chunk given in host memory
+  cudaEvent_t noise_ev = nullptr;     // its upload has left the staging
   // bookkeeping (host, exact)
   long long step = 0, next_id = 0, head_id = 0, ready_lo = 0;
   bool closed = false;

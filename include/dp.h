@@ -193,11 +193,10 @@ DP_API dp_status dp_queue_init(dp_model* m, const dp_queue_config* qc, const flo
  * part of the step enqueued: the queue must then be destroyed (or reloaded
  * with dp_queue_load_state).  A queue is not safe to use from several host
  * threads at once.
- * Ownership: the step is asynchronous on the model's stream.  A device buffer,
- * or a page-locked host buffer, is read when the stream reaches the push, so
- * the caller must not overwrite it before the step completes (dp_queue_sync or
- * a later event on the stream); a pageable host buffer is copied before the
- * call returns. */
+ * Ownership: a host `new_chunk_noise` (pageable or page-locked) is copied into
+ * the queue's pinned staging before the call returns and may be reused at
+ * once; a device one is read in stream order, so it must not be overwritten
+ * before the step has run (dp_queue_sync, or a later event on the stream). */
 DP_API dp_status dp_queue_step(dp_queue* q, const float* new_chunk_noise, dp_loc loc);
 
 /* Copies the oldest ready chunk ([C][F][H][W] fp32) to `out` at `loc` and

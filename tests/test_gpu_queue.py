@@ -119,6 +119,39 @@ def test_degenerate_queues_match_oracle(precision, T, N):
     model.close()
 
 
+def test_host_noise_buffer_is_free_when_step_returns():
+    """One page-locked host buffer carries every pushed chunk: it is refilled
+    with the next chunk's noise (and poisoned in between) as soon as each step
+    returns, while the queue's stream may still be busy; the popped chunks
+    must still match the oracle stream (fp32, 1e-4)."""
+    w = synth.WORKLOADS["tiny_fp32"]
+    m, q = w.model, w.queue
+    model, queue, p, text = make(w, "fp32")
+    noise = [synth.make_noise(m, q, k) for k in range(q.n_chunks)]
+    fn = dit.make_velocity_fn(p, text, m, q.T)
+    ready, traces = fifo.run_stream(fn, lambda k: noise[k], q.T, q.n_chunks)
+    buf = torch.empty(q.chunk_shape(m), dtype=torch.float32).pin_memory()
+    out = np.empty(q.chunk_shape(m), np.float32)
+    got = {}
+    for tr in traces:
+        if tr.step < q.n_chunks:
+            buf.copy_(torch.from_numpy(noise[tr.step]))
+            queue.step(buf)
+            buf.fill_(float("nan"))
+        else:
+            queue.step(None)
+        while True:
+            st, cid = queue.try_pop(out)
+            if st != 0:
+                break
+            got[cid] = out.copy()
+    queue.sync()
+    assert sorted(got) == list(range(q.n_chunks))
+    for k, ref in ready:
+        assert rel_l2(got[k], ref) <= 1e-4, (k, rel_l2(got[k], ref))
+    model.close()
+
+
 def test_invalid_configurations_are_rejected():
     import ctypes as C
     from chunked_fifo_denoising_b200 import Model, Queue, DPError
