@@ -1056,6 +1056,7 @@ dp_status dp_queue_inspect(const dp_queue* q, dp_queue_info* info, long long* id
 dp_status dp_queue_read_latents(dp_queue* q, float* out, int n, dp_loc loc) {
   clear_error();
   if (!q || !out) return fail(DP_ERR_INVALID_ARG, "NULL argument");
+  if (loc != DP_LOC_DEVICE && loc != DP_LOC_HOST) return fail(DP_ERR_INVALID_ARG, "bad location");
   if (n != (int)q->levels.size())
     return fail(DP_ERR_INVALID_ARG, "queue holds %d chunks, asked for %d", (int)q->levels.size(), n);
   cudaStream_t s = q->m->stream;
@@ -1132,6 +1133,7 @@ dp_status dp_queue_load_state(dp_queue* q, long long step, long long n_pushed, i
 dp_status dp_queue_read_pred_kv(dp_queue* q, float* out, dp_loc loc, long long* chunk_id) {
   clear_error();
   if (!q || !out) return fail(DP_ERR_INVALID_ARG, "NULL argument");
+  if (loc != DP_LOC_DEVICE && loc != DP_LOC_HOST) return fail(DP_ERR_INVALID_ARG, "bad location");
   dp_model* m = q->m;
   cudaStream_t s = m->stream;
   const size_t blk = (size_t)q->Lc * m->d;

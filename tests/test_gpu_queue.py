@@ -181,6 +181,13 @@ def test_invalid_configurations_are_rejected():
     with pytest.raises(DPError):        # read_latents with a wrong count
         queue.read_latents(3)
     assert B.dp_queue_step(None, None, 0) == B.DP_ERR_INVALID_ARG
+    # a location that is neither host nor device is rejected before any copy
+    buf = np.empty(q.chunk_numel(m) * 4, np.float32)
+    assert B.dp_queue_read_latents(queue.handle, buf.ctypes.data, 0, 7) == B.DP_ERR_INVALID_ARG
+    cid = C.c_longlong()
+    assert B.dp_queue_read_pred_kv(queue.handle, buf.ctypes.data, 7, cid) == B.DP_ERR_INVALID_ARG
+    assert B.dp_queue_step(queue.handle, buf.ctypes.data, 7) == B.DP_ERR_INVALID_ARG
+    assert B.dp_queue_pop(queue.handle, buf.ctypes.data, 7, cid) == B.DP_ERR_INVALID_ARG
     model.close()
 
 
