@@ -12,7 +12,9 @@
  * They allocate nothing.  Errors: DP_ERR_INVALID_ARG for a NULL pointer, a
  * non-positive or unsupported size, a misaligned pointer or leading dimension
  * (the bf16 tensor-core paths need 16-byte aligned rows); DP_ERR_CUDA if the
- * launch fails.  The message is in dp_last_error().
+ * launch fails.  The message is in dp_last_error().  The extent behind a raw
+ * pointer cannot be checked: the caller guarantees that every buffer holds the
+ * rows and leading dimension its sizes imply.
  *
  * Method source: the DualParal write-up "双重并行：让AI视频生成突破时长限制…"
  * (techwalker.com) §三: self-attention of a chunk reads its neighbour's cached
