@@ -45,3 +45,28 @@ def test_param_numel_and_config_errors():
     bad.n_heads = 7
     assert B.dp_param_numel(bad, 0, n) == B.DP_ERR_INVALID_ARG
     assert "n_heads" in B.dp_last_error() or "head" in B.dp_last_error()
+
+
+def test_binding_marshals_buffers_by_location_and_rejects_bad_ones():
+    """The binding only marshals: numpy arrays and CPU tensors are host buffers,
+    CUDA tensors device buffers; wrong dtypes or layouts are refused before any
+    call into the library."""
+    import numpy as np
+    import torch
+    from chunked_fifo_denoising_b200 import _binding as B
+    from chunked_fifo_denoising_b200.queue import _ptr
+    a = np.zeros((3, 4), np.float32)
+    assert _ptr(a) == (a.ctypes.data, B.DP_LOC_HOST)
+    t = torch.zeros(3, 4)
+    assert _ptr(t) == (t.data_ptr(), B.DP_LOC_HOST)
+    assert _ptr(None) == (None, B.DP_LOC_DEVICE)
+    with pytest.raises(TypeError):
+        _ptr(np.zeros(4, np.float64))
+    with pytest.raises(ValueError):
+        _ptr(np.zeros((4, 4), np.float32)[:, ::2])
+    with pytest.raises(TypeError):
+        _ptr(torch.zeros(4, dtype=torch.float16))
+    with pytest.raises(ValueError):
+        _ptr(torch.zeros(4, 4).t())
+    with pytest.raises(TypeError):
+        _ptr([1.0, 2.0])
