@@ -114,6 +114,7 @@ _SIGS = {
     "dp_op_gemm": (C.c_int, [C.POINTER(dp_gemm_args), C.c_void_p]),
     "dp_op_attention": (C.c_int, [C.POINTER(dp_attn_args), C.c_void_p]),
     "dp_op_layernorm_mod": (C.c_int, [C.POINTER(dp_ln_args), C.c_void_p]),
+    "dp_op_ln_gemm_noalloc": (C.c_int, [C.POINTER(dp_ln_args), C.POINTER(dp_gemm_args), C.c_void_p]),
     "dp_op_check": (C.c_int, [C.c_void_p]),
     "dp_op_selftest_timeout": (C.c_int, [C.c_void_p]),
 }
@@ -180,5 +181,6 @@ def dp_last_error(): return lib().dp_last_error().decode(errors="replace")
 def dp_op_gemm(args, stream): return _call("dp_op_gemm", C.byref(args), stream)
 def dp_op_attention(args, stream): return _call("dp_op_attention", C.byref(args), stream)
 def dp_op_layernorm_mod(args, stream): return _call("dp_op_layernorm_mod", C.byref(args), stream)
+def dp_op_ln_gemm_noalloc(ln, gemm, stream): return _call("dp_op_ln_gemm_noalloc", C.byref(ln), C.byref(gemm), stream)
 def dp_op_check(stream): return _call("dp_op_check", stream)
 def dp_op_selftest_timeout(stream): return _call("dp_op_selftest_timeout", stream)

@@ -104,6 +104,35 @@ typedef struct {
 } dp_ln_args;
 DP_API dp_status dp_op_layernorm_mod(const dp_ln_args* a, void* stream);
 
+/* The modulated projection of a DiT block, LN + adaLN (as dp_op_layernorm_mod)
+ * followed by the GEMM that reads its output (as dp_op_gemm), for callers that
+ * may not allocate device memory.  This is a library convenience: the
+ * DualParal write-up has no counterpart to it.
+ *
+ * Who needs it: code that runs inside a host framework whose allocator owns
+ * all device memory (memory taken with cudaMalloc behind its back can make it
+ * run out, and cudaMalloc/cudaFree synchronise the device), and services that
+ * plan their memory at start-up and must not allocate on the request path.
+ * Such callers own their inputs and outputs but have nowhere to put the
+ * normalised rows that pass from one kernel to the next.  This call keeps
+ * them in one static device array of 32 MiB that the library holds on every
+ * GPU that loads it, until the process exits.  It calls no cudaMalloc,
+ * cudaFree or allocating library routine.
+ *
+ * Arguments: `ln` and `gemm` as for the two calls above, with ln->out and
+ * gemm->A NULL (the scratch takes their place, packed with leading dimension
+ * ln->d); gemm->M == ln->M, gemm->K == ln->d and ln->out_dtype == gemm->dtype.
+ * Limit: ln->M * ln->d * (2 for bf16, 4 for f32) <= 32 MiB, else
+ * DP_ERR_INVALID_ARG with the sizes in dp_last_error().  Other errors as for
+ * dp_op_layernorm_mod and dp_op_gemm.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  Every call, on any stream, uses the same array, and each call
+ * overwrites the rows it uses before reading them, so nothing needs clearing;
+ * but calls whose work overlaps on the GPU (other streams, other host threads)
+ * race on it: order them on one stream. */
+DP_API dp_status dp_op_ln_gemm_noalloc(const dp_ln_args* ln, const dp_gemm_args* gemm, void* stream);
+
 /* Exercises the bounded-wait failure path: launches one block that waits on
  * an mbarrier nothing arrives at, gives up after the kernels' wait limit
  * (2 s), sets the status word and returns; nothing faults.  A following
