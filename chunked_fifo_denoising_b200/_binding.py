@@ -98,6 +98,7 @@ _SIGS = {
     "dp_queue_close": (C.c_int, [C.c_void_p]),
     "dp_queue_set_noise_pool": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int]),
     "dp_queue_sync": (C.c_int, [C.c_void_p]),
+    "dp_queue_selftest_timeout": (C.c_int, [C.c_void_p]),
     "dp_queue_inspect": (C.c_int, [C.c_void_p, C.POINTER(dp_queue_info), C.c_void_p, C.c_void_p,
                                    C.c_void_p, C.c_void_p, C.c_int]),
     "dp_queue_read_latents": (C.c_int, [C.c_void_p, C.c_void_p, C.c_int, C.c_int]),
@@ -169,6 +170,7 @@ def dp_queue_pop(q, out, loc, cid): return _call("dp_queue_pop", q, out, loc, C.
 def dp_queue_close(q): return _call("dp_queue_close", q)
 def dp_queue_set_noise_pool(q, pool, loc): return _call("dp_queue_set_noise_pool", q, pool, loc)
 def dp_queue_sync(q): return _call("dp_queue_sync", q)
+def dp_queue_selftest_timeout(q): return _call("dp_queue_selftest_timeout", q)
 def dp_queue_inspect(q, info, ids, levels, slots, positions, cap): return _call("dp_queue_inspect", q, C.byref(info), ids, levels, slots, positions, cap)
 def dp_queue_read_latents(q, out, n, loc): return _call("dp_queue_read_latents", q, out, n, loc)
 def dp_queue_load_state(q, step, n_pushed, n, lat, kv, loc): return _call("dp_queue_load_state", q, step, n_pushed, n, lat, kv, loc)

@@ -722,6 +722,19 @@ static dp_status upload_tables(dp_queue* q, const Plan& pl) {
   return DP_OK;
 }
 
+// Reads and clears the model's device status word (the stream must have been
+// synchronised): DP_ERR_KERNEL if a kernel gave up a bounded wait since the
+// last check.
+static dp_status check_status_word(dp_model* m) {
+  int word = 0;
+  DP_CK(cudaMemcpy(&word, m->status.p, sizeof(int), cudaMemcpyDeviceToHost));
+  if (word != 0) {
+    DP_CK(cudaMemset(m->status.p, 0, 256));
+    return fail(DP_ERR_KERNEL, "a kernel gave up a bounded wait (status word 0x%x)", word);
+  }
+  return DP_OK;
+}
+
 static void free_queue(dp_queue* q) {
   DevBuf* bufs[] = {&q->ring, &q->x, &q->h, &q->qkv, &q->attn, &q->u, &q->textkv, &q->cache[0],
                     &q->cache[1], &q->modtab, &q->hmod, &q->d_sel, &q->d_slot, &q->d_dsig,
@@ -987,9 +1000,14 @@ dp_status dp_queue_pop(dp_queue* q, float* out, dp_loc loc, long long* chunk_id)
   const float* slot = q->ring.as<float>() + (size_t)(q->ready_lo % q->n_slots) * q->chunk_numel;
   DP_CK(cudaMemcpyAsync(out, slot, (size_t)q->chunk_numel * 4,
                         loc == DP_LOC_HOST ? cudaMemcpyDeviceToHost : cudaMemcpyDeviceToDevice, s));
-  if (loc == DP_LOC_HOST) DP_CK(cudaStreamSynchronize(s));
   if (chunk_id) *chunk_id = q->ready_lo;
   q->ready_lo += 1;
+  if (loc == DP_LOC_HOST) {
+    // the copy has been waited for anyway: report a kernel that gave up a
+    // bounded wait (and skipped its work) instead of returning its result as good
+    DP_CK(cudaStreamSynchronize(s));
+    DP_TRY(check_status_word(q->m));
+  }
   return DP_OK;
 }
 
@@ -1017,12 +1035,14 @@ dp_status dp_queue_sync(dp_queue* q) {
   if (!q) return fail(DP_ERR_INVALID_ARG, "NULL queue");
   dp_model* m = q->m;
   DP_CK(cudaStreamSynchronize(m->stream));
-  int word = 0;
-  DP_CK(cudaMemcpy(&word, m->status.p, sizeof(int), cudaMemcpyDeviceToHost));
-  if (word != 0) {
-    DP_CK(cudaMemset(m->status.p, 0, 256));
-    return fail(DP_ERR_KERNEL, "a kernel gave up a bounded wait (status word 0x%x)", word);
-  }
+  return check_status_word(m);
+}
+
+dp_status dp_queue_selftest_timeout(dp_queue* q) {
+  clear_error();
+  if (!q) return fail(DP_ERR_INVALID_ARG, "NULL queue");
+  cudaError_t err = selftest_timeout(q->m->status.as<int>(), q->m->stream);
+  if (err != cudaSuccess) return fail(DP_ERR_CUDA, "self test launch: %s", cudaGetErrorString(err));
   return DP_OK;
 }
 
@@ -1077,6 +1097,10 @@ dp_status dp_queue_load_state(dp_queue* q, long long step, long long n_pushed, i
   const int T = q->qc.T;
   if (n < 0 || n > T || n_pushed < n || step < n_pushed || (q->qc.n_chunks >= 0 && n_pushed > q->qc.n_chunks))
     return fail(DP_ERR_INVALID_ARG, "inconsistent state (step %lld, pushed %lld, n %d)", step, n_pushed, n);
+  // Every check comes before the first copy, so a rejected state leaves the
+  // queue as it was.  A FIFO stream pushes chunk k at step k and chunk k
+  // leaves after step k + T - 1; before step `step` the queued chunks are
+  // therefore exactly [max(0, step - T + 1), n_pushed).
   const long long head = n_pushed - n;
   std::deque<int> lv;
   for (long long k = head; k < n_pushed; ++k) {
@@ -1084,7 +1108,18 @@ dp_status dp_queue_load_state(dp_queue* q, long long step, long long n_pushed, i
     if (j < 1 || j > T) return fail(DP_ERR_INVALID_ARG, "chunk %lld would be at level %lld", k, j);
     lv.push_back((int)j);
   }
+  if (head != std::max(0LL, step - T + 1) && !(n == 0 && head <= step - T + 1))
+    return fail(DP_ERR_INVALID_ARG,
+                "chunks [%lld, %lld) at step %lld: chunk %lld has not left the queue yet", head, n_pushed,
+                step, head - 1);
+  // Pushes stop when n_chunks are in, or when the stream was closed; a state
+  // past its last push (step > n_pushed) with pushes still allowed by n_chunks
+  // is a closed stream, and is restored closed.
+  const bool closed = step > n_pushed;
   dp_model* m = q->m;
+  const size_t blk = (size_t)q->Lc * m->d;
+  if (pred_kv && loc == DP_LOC_HOST && blk * 4 > m->staging.bytes)
+    return fail(DP_ERR_INVALID_ARG, "predecessor block of %zu floats larger than the staging buffer", blk);
   cudaStream_t s = m->stream;
   const cudaMemcpyKind kind = loc == DP_LOC_HOST ? cudaMemcpyHostToDevice : cudaMemcpyDeviceToDevice;
   for (int i = 0; i < n; ++i) {
@@ -1092,19 +1127,13 @@ dp_status dp_queue_load_state(dp_queue* q, long long step, long long n_pushed, i
     DP_CK(cudaMemcpyAsync(slot, latents + (size_t)i * q->chunk_numel, (size_t)q->chunk_numel * 4, kind, s));
   }
   if (pred_kv) {
-    const size_t cnt = (size_t)m->L * q->Lc * 2 * m->d;
-    // staging is a model buffer sized for the largest parameter; use it in pieces
-    const size_t per = m->staging.bytes / 4;
-    const float* src = pred_kv;
-    size_t done = 0;
-    // fp32 source layout [L][2][Lc][d] -> cache layout [L][Lc][2d]
+    // fp32 source layout [L][2][Lc][d] -> cache layout [L][Lc][2d]; host
+    // blocks pass through the model's staging buffer one at a time
     for (int l = 0; l < m->L; ++l) {
       for (int kv = 0; kv < 2; ++kv) {
-        const size_t blk = (size_t)q->Lc * m->d;
-        const float* part = src + ((size_t)l * 2 + kv) * blk;
+        const float* part = pred_kv + ((size_t)l * 2 + kv) * blk;
         const float* dsrc = part;
         if (loc == DP_LOC_HOST) {
-          if (blk > per) return fail(DP_ERR_INVALID_ARG, "predecessor block larger than staging");
           DP_CK(cudaMemcpyAsync(m->staging.p, part, blk * 4, cudaMemcpyHostToDevice, s));
           dsrc = m->staging.as<float>();
         }
@@ -1112,11 +1141,8 @@ dp_status dp_queue_load_state(dp_queue* q, long long step, long long n_pushed, i
                     ((size_t)l * q->Lc * 2 * m->d + (size_t)kv * m->d) * m->act_size();
         DP_CK(copy_rows(dsrc, 1, m->d, dst, m->f32 ? 1 : 0, 2 * m->d, q->Lc, m->d, s));
         if (loc == DP_LOC_HOST) DP_CK(cudaStreamSynchronize(s));
-        done += blk;
       }
     }
-    (void)cnt;
-    (void)done;
     q->cache_id = head - 1;
   } else {
     q->cache_id = -1;
@@ -1127,6 +1153,7 @@ dp_status dp_queue_load_state(dp_queue* q, long long step, long long n_pushed, i
   q->head_id = head;
   q->ready_lo = head;
   q->levels = lv;
+  q->closed = closed;
   return DP_OK;
 }
 

@@ -72,6 +72,9 @@ dp_status dp_op_attention(const dp_attn_args* a, void* stream) {
     return fail(DP_ERR_INVALID_ARG, "bad predecessor buffer");
   if ((a->pred_in_batch || a->succ_in_batch) && a->kv_chunk_rows <= 0)
     return fail(DP_ERR_INVALID_ARG, "pred_in_batch / succ_in_batch need per-chunk keys");
+  if (a->kv_chunk_rows > 0 && a->Lk > a->kv_chunk_rows)
+    return fail(DP_ERR_INVALID_ARG, "Lk %d exceeds kv_chunk_rows %lld: a chunk's keys would run into the next chunk's",
+                a->Lk, a->kv_chunk_rows);
   AttnParams p;
   memset(&p, 0, sizeof(p));
   p.f32 = a->dtype == DP_DT_F32;
@@ -112,7 +115,7 @@ dp_status dp_op_attention(const dp_attn_args* a, void* stream) {
 
 dp_status dp_op_selftest_timeout(void* stream) {
   clear_error();
-  cudaError_t err = selftest_timeout(static_cast<cudaStream_t>(stream));
+  cudaError_t err = selftest_timeout(nullptr, static_cast<cudaStream_t>(stream));
   if (err != cudaSuccess) return fail(DP_ERR_CUDA, "self test launch: %s", cudaGetErrorString(err));
   return DP_OK;
 }

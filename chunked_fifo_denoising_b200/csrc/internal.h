@@ -116,8 +116,9 @@ cudaError_t normal_fill(unsigned long long seed, unsigned long long a, unsigned 
 
 // Device status word of kernels launched from the single-kernel entry points.
 int* op_status_word();
-// A kernel whose only mbarrier wait times out (failure-path self test).
-cudaError_t selftest_timeout(cudaStream_t s);
+// A kernel whose only mbarrier wait times out (failure-path self test); it
+// sets `status` (NULL: the status word of the single-kernel entry points).
+cudaError_t selftest_timeout(int* status, cudaStream_t s);
 
 // slot [C][F][HW] <- pool [2F][C][HW]: frame f of the chunk is pool frame src[f]
 struct PoolGather { int src[64]; };

@@ -497,8 +497,8 @@ __global__ void selftest_timeout_kernel(int* status) {
   __syncthreads();
 }
 
-cudaError_t selftest_timeout(cudaStream_t s) {
-  int* status = op_status_word();
+cudaError_t selftest_timeout(int* status, cudaStream_t s) {
+  if (!status) status = op_status_word();
   if (!status) return cudaErrorInvalidValue;
   selftest_timeout_kernel<<<1, 32, 0, s>>>(status);
   return cudaGetLastError();

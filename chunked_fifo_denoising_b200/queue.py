@@ -146,6 +146,10 @@ class Queue:
     def sync(self):
         return B.check(B.dp_queue_sync(self.handle), "dp_queue_sync")
 
+    def selftest_timeout(self):
+        """Enqueues the bounded-wait self test on the queue's stream."""
+        B.check(B.dp_queue_selftest_timeout(self.handle), "dp_queue_selftest_timeout")
+
     def inspect(self):
         info = B.dp_queue_info()
         cap = self.qc.T

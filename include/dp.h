@@ -161,6 +161,8 @@ DP_API dp_status dp_set_allocator(dp_alloc_fn alloc, dp_free_fn free_fn, void* c
 DP_API dp_status dp_param_numel(const dp_model_config* cfg, dp_param id, long long* numel);
 
 /* Creates a model on the current CUDA device and allocates its weights.
+ * The model is the per-chunk-timestep DiT of the write-up's section 一 (every
+ * chunk of the queue carries its own noise level into the block's adaLN).
  * `cuda_stream` is a cudaStream_t (NULL = legacy default stream) on which all
  * later work of this model and its queues runs. */
 DP_API dp_status dp_model_create(const dp_model_config* cfg, void* cuda_stream, dp_model** out);
@@ -171,7 +173,10 @@ DP_API dp_status dp_model_create(const dp_model_config* cfg, void* cuda_stream, 
 DP_API dp_status dp_model_set_param(dp_model* m, dp_param id, int layer, const float* src,
                              long long numel, dp_loc loc);
 
-/* Starts a queue: allocates the latent ring (T + ready_capacity chunk slots),
+/* Starts a queue (section 二: a FIFO of chunks, levels T at the tail down to 1
+ * at the head; section 三: the prompt's cross-attention K/V serve every chunk
+ * and every step, so they are projected once, here).
+ * Allocates the latent ring (T + ready_capacity chunk slots),
  * the activations for T chunks and the double-buffered predecessor K/V cache;
  * projects the prompt `text` ([text_len][text_in_dim] fp32) to the per-layer
  * cross-attention K/V once; builds the per-level modulation tables.  The queue
@@ -179,7 +184,11 @@ DP_API dp_status dp_model_set_param(dp_model* m, dp_param id, int layer, const f
 DP_API dp_status dp_queue_init(dp_model* m, const dp_queue_config* qc, const float* text,
                         dp_loc text_loc, dp_queue** out);
 
-/* One queue step.  If a chunk is due (fewer than n_chunks pushed and the queue
+/* One queue step (section 二: every queued chunk is denoised once and moves one
+ * place toward the head, a noisy chunk enters at the tail, the clean one
+ * leaves at the head; section 三: a chunk's self-attention reads its
+ * neighbour's K/V next to its own, never a concatenated input).
+ * If a chunk is due (fewer than n_chunks pushed and the queue
  * not closed), it is pushed at the tail at level T first, its latent taken
  * from `new_chunk_noise` ([C][F][H][W] fp32 at `loc`), or drawn N(0,1) by the
  * internal generator when `new_chunk_noise` is NULL.  Then every queued chunk
@@ -199,14 +208,21 @@ DP_API dp_status dp_queue_init(dp_model* m, const dp_queue_config* qc, const flo
  * before the step has run (dp_queue_sync, or a later event on the stream). */
 DP_API dp_status dp_queue_step(dp_queue* q, const float* new_chunk_noise, dp_loc loc);
 
-/* Copies the oldest ready chunk ([C][F][H][W] fp32) to `out` at `loc` and
- * frees its slot; `chunk_id` (may be NULL) receives its id.  Chunk ids pop in
- * strictly increasing order.  DP_ERR_EMPTY if none is ready.  A host `out` is
- * complete when the call returns (it waits for the stream); a device `out` is
- * written in stream order. */
+/* Pop at the head of the FIFO (section 二: the clean chunk leaves for the
+ * decoder).  Copies the oldest ready chunk ([C][F][H][W] fp32) to `out` at
+ * `loc` and frees its slot; `chunk_id` (may be NULL) receives its id.  Chunk
+ * ids pop in strictly increasing order.  DP_ERR_EMPTY if none is ready.  A
+ * host `out` is complete when the call returns: the call waits for the stream
+ * and then checks the device status word, returning DP_ERR_KERNEL (the chunk
+ * is still consumed and `chunk_id` set) if a kernel gave up a bounded wait
+ * since the last check, because the chunk may then hold skipped work; reload
+ * the queue (dp_queue_load_state) or destroy it.  A device `out` is written in
+ * stream order and not checked: call dp_queue_sync for that. */
 DP_API dp_status dp_queue_pop(dp_queue* q, float* out, dp_loc loc, long long* chunk_id);
 
-/* Replaces the coordinated-noise pool (noise_mode 1) with `pool`
+/* Coordinated noise initialisation (section 三: a new chunk's noise comes from
+ * a pool, avoiding the frames its neighbour used, shuffled).
+ * Replaces the coordinated-noise pool (noise_mode 1) with `pool`
  * ([2F][C][H][W] fp32 at `loc`).  By default the pool is drawn N(0,1) on the
  * device at dp_queue_init (frame b from stream (seed, 1003, b)).  Synchronous. */
 DP_API dp_status dp_queue_set_noise_pool(dp_queue* q, const float* pool, dp_loc loc);
@@ -218,7 +234,15 @@ DP_API dp_status dp_queue_close(dp_queue* q);
  * DP_ERR_KERNEL if a kernel gave up a bounded wait since the last check. */
 DP_API dp_status dp_queue_sync(dp_queue* q);
 
-/* Bookkeeping of the NEXT step, as dp_queue_step would run it now (including
+/* Exercises the failure path of the queue's bounded waits: enqueues on the
+ * queue's stream one block that waits on an mbarrier nothing arrives at, gives
+ * up after the kernels' wait limit (2 s), sets the queue's status word and
+ * returns; nothing faults and the queue's data is untouched.  The next
+ * dp_queue_sync or host dp_queue_pop then reports DP_ERR_KERNEL once. */
+DP_API dp_status dp_queue_selftest_timeout(dp_queue* q);
+
+/* Bookkeeping of the FIFO (section 二) for the NEXT step, as dp_queue_step
+ * would run it now (including
  * the chunk it would push).  Arrays hold up to `cap` entries, head first:
  * chunk ids, levels (1..T), ring slots and queue positions (level - 1).
  * head_pred: 0 = none (head is chunk 0), 2 = persisted K/V of the chunk that
@@ -249,7 +273,16 @@ DP_API dp_status dp_queue_read_latents(dp_queue* q, float* out, int n, dp_loc lo
  * `loc`) and levels taken from the FIFO schedule; `pred_kv` ([n_layers][2]
  * [tokens_per_chunk][dim] fp32, K then V per layer, or NULL) are the persisted
  * self-attention K/V of chunk n_pushed - n - 1.  No chunk is ready after it.
- * Synchronous.  For per-step parity tests and resuming a checkpoint. */
+ * Synchronous.  For per-step parity tests and resuming a checkpoint.
+ * Only states a FIFO stream reaches are accepted (DP_ERR_INVALID_ARG
+ * otherwise, with the queue unchanged): chunk k is pushed at step k and leaves
+ * after step k + T - 1, so before `step` the queued chunks must be exactly
+ * [max(0, step - T + 1), n_pushed), with step >= n_pushed.  A state with
+ * step > n_pushed has stopped pushing: it is restored closed (as after
+ * dp_queue_close); with step == n_pushed the queue is open and pushes while
+ * n_chunks allows (call dp_queue_close after loading to end it there).  Leaving
+ * `pred_kv` NULL while the head chunk has a predecessor makes the next step
+ * fail with DP_ERR_STATE. */
 DP_API dp_status dp_queue_load_state(dp_queue* q, long long step, long long n_pushed, int n,
                               const float* latents, const float* pred_kv, dp_loc loc);
 

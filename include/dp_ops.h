@@ -43,8 +43,9 @@ typedef enum {
 
 /* out/resid = epilogue(A[M][K] . W[N][K]^T + bias).
  * dtype: of A, W and (STORE/GELU) out.  bf16 runs on the tcgen05 tensor cores
- * with fp32 accumulation (needs K % 64 == 0, N % 16 == 0, lda and ldo
- * multiples of 8); f32 runs FFMA.
+ * with fp32 accumulation (needs K % 64 == 0, N % 32 == 0, lda and ldo
+ * multiples of 8, 16-byte aligned pointers, and for a cache copy ldc % 8 == 0
+ * and cache_col0 % 32 == 0); f32 runs FFMA.
  * gate(r, c) = gate[sel(r / rows_per_chunk) * gate_stride + c] with
  * sel(i) = chunk_sel[i] (device int array) or i when chunk_sel is NULL.
  * The optional cache copy also writes, for rows r in
@@ -77,7 +78,10 @@ DP_API dp_status dp_op_gemm(const dp_gemm_args* a, void* stream);
  *   - if succ_in_batch and c < n_chunks - 1: the own keys of chunk c + 1.
  * Queries of chunk c are rows [c * Lq, (c + 1) * Lq) of q.  Head h uses
  * columns [h * head_dim, (h + 1) * head_dim) of q, k, v and out.
- * bf16 requires head_dim 64 or 128 (tcgen05 path); f32 requires head_dim <= 128. */
+ * With per-chunk keys (kv_chunk_rows > 0), Lk <= kv_chunk_rows.
+ * bf16 requires head_dim 64 or 128 (tcgen05 path), leading dimensions that
+ * are multiples of 8 and 16-byte aligned pointers; f32 requires head_dim in
+ * {16, 32, 64, 128}. */
 typedef struct {
   dp_dtype dtype;
   int n_chunks, Lq, n_heads, head_dim;

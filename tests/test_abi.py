@@ -70,3 +70,29 @@ def test_binding_marshals_buffers_by_location_and_rejects_bad_ones():
         _ptr(torch.zeros(4, 4).t())
     with pytest.raises(TypeError):
         _ptr([1.0, 2.0])
+
+
+def test_attention_rejects_keys_running_into_the_next_chunk():
+    """With per-chunk keys, Lk > kv_chunk_rows would read the next chunk's rows
+    (and the f32 and bf16 paths would disagree past the last chunk): refused
+    by the argument checks, before anything reaches the device."""
+    from chunked_fifo_denoising_b200 import _binding as B
+    a = B.dp_attn_args()
+    a.dtype, a.n_chunks, a.Lq, a.n_heads, a.head_dim = B.DP_DT_F32, 2, 8, 1, 16
+    a.q = a.k = a.v = a.out = 4096          # never dereferenced: the call fails first
+    a.ldq = a.ldkv = a.ldo = 16
+    a.kv_chunk_rows, a.Lk, a.pred_in_batch = 8, 9, 1
+    assert B.dp_op_attention(a, None) == B.DP_ERR_INVALID_ARG
+    assert "kv_chunk_rows" in B.dp_last_error()
+
+
+def test_noalloc_projection_refuses_oversized_rows_before_any_device_work():
+    from chunked_fifo_denoising_b200 import _binding as B
+    ln, g = B.dp_ln_args(), B.dp_gemm_args()
+    ln.out_dtype = g.dtype = B.DP_DT_BF16
+    ln.x, ln.ldx = 4096, 6144
+    ln.M = g.M = 4096
+    ln.d = g.K = 6144                       # 4096 x 6144 bf16 = 48 MiB > 32 MiB
+    g.W, g.N, g.out, g.ldo = 4096, 64, 8192, 64
+    assert B.dp_op_ln_gemm_noalloc(ln, g, None) == B.DP_ERR_INVALID_ARG
+    assert "static scratch" in B.dp_last_error()

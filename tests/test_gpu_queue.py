@@ -9,7 +9,10 @@ float64 oracle on identical seeded inputs:
   2e-2 on the velocity of every chunk, on the persisted K/V and on the latents
   (small workload; Wan-1.3B shapes with two layers; Wan-14B shapes with one
   layer; the bidirectional neighbourhood; QK RMSNorm with rotary positions);
-* resuming from latents and persisted K/V read mid-stream is bit-exact;
+* resuming from latents and persisted K/V read mid-stream is bit-exact, and
+  matches the oracle (whole fp32 stream; one bf16 step from the checkpoint);
+* load_state accepts only states a FIFO stream reaches; a host pop reports a
+  kernel that gave up a bounded wait;
 * error codes, the internal noise generator, flat device memory.
 """
 import numpy as np
@@ -332,6 +335,164 @@ def test_checkpoint_resume_is_bit_exact():
     assert sorted(got_a) == sorted(got_b) and len(got_a) > 0
     for k in got_a:
         assert np.array_equal(got_a[k], got_b[k]), k
+    model.close()
+
+
+def test_resume_matches_the_oracle_stream():
+    """fp32 validation mode, tiny workload: a checkpoint read mid-stream (head
+    chunk with a persisted predecessor, pushes still due) and loaded into a new
+    queue finishes the stream; every chunk popped before and after the
+    checkpoint matches the oracle's unbroken stream (relative L2 1e-4)."""
+    from chunked_fifo_denoising_b200 import Queue
+    w = synth.WORKLOADS["tiny_fp32"]
+    m, q = w.model, w.queue
+    N, T, s_ck = q.n_chunks, q.T, 5
+    model, qa, p, text = make(w, "fp32")
+    noise = [synth.make_noise(m, q, k) for k in range(N)]
+    out = np.empty(q.chunk_shape(m), np.float32)
+    got = {}
+
+    def drain(qq):
+        while True:
+            st, cid = qq.try_pop(out)
+            if st != 0:
+                return
+            got[cid] = out.copy()
+    for s in range(s_ck):
+        qa.step(noise[s])
+        drain(qa)
+    info = qa.inspect()
+    n_pushed = info["next_push_id"]
+    assert info["step"] == s_ck and n_pushed == s_ck          # pushes still due
+    n_q = info["n"] - 1
+    lat = qa.read_latents(n_q)
+    kv, kv_id = qa.read_pred_kv()
+    assert kv_id == n_pushed - n_q - 1 >= 0                  # the head has a persisted predecessor
+    qa.close()
+    qb = Queue(model, text, T, q.frames_per_chunk, q.lat_h, q.lat_w, N)
+    qb.load_state(s_ck, n_pushed, lat, kv)
+    assert qb.inspect()["ids"] == info["ids"] and qb.inspect()["levels"] == info["levels"]
+    s = s_ck
+    while qb.try_step(noise[s] if s < N else None) == 0:
+        s += 1
+        drain(qb)
+    drain(qb)
+    assert s == N + T - 1
+    fn = dit.make_velocity_fn(p, text, m, T)
+    ready, _ = fifo.run_stream(fn, lambda k: noise[k], T, N)
+    assert sorted(got) == list(range(N))
+    for k, ref in ready:
+        assert rel_l2(got[k], ref) <= 1e-4, k
+    model.close()
+
+
+def test_resumed_bf16_step_matches_the_oracle_step():
+    """bf16, small workload with two layers: the checkpoint of a GPU stream,
+    loaded into a new queue, takes one step (with a push) that matches the
+    oracle's step from the same checkpoint within relative L2 2e-2 on every
+    chunk's latent and on the newly persisted K/V."""
+    from chunked_fifo_denoising_b200 import Queue
+    w = synth.truncated(synth.WORKLOADS["small_bf16"], 2)
+    m, q = w.model, w.queue
+    N, T, s_ck = 14, q.T, 12
+    model, qa, p, text = make(w, "bf16", n_chunks=N)
+    noise = [synth.make_noise(m, q, k) for k in range(N)]
+    out = np.empty(q.chunk_shape(m), np.float32)
+    for s in range(s_ck):
+        qa.step(noise[s])
+        while qa.try_pop(out)[0] == 0:
+            pass
+    info = qa.inspect()
+    n_pushed, n_q = info["next_push_id"], info["n"] - 1
+    lat = qa.read_latents(n_q)
+    kv, kv_id = qa.read_pred_kv()
+    head = n_pushed - n_q
+    assert kv_id == head - 1 >= 0 and info["levels"][0] == 1
+    qa.close()
+    qb = Queue(model, text, T, q.frames_per_chunk, q.lat_h, q.lat_w, N)
+    qb.load_state(s_ck, n_pushed, lat, kv)
+    qb.step(noise[n_pushed])
+    qb.sync()
+    popped = np.empty(q.chunk_shape(m), np.float32)
+    assert qb.pop(popped) == head
+    rest = qb.read_latents(n_q)              # the chunks after the head, plus the one pushed
+    new_kv, new_id = qb.read_pred_kv()
+    assert new_id == head
+    fn = dit.make_velocity_fn(p, text, m, T)
+    st = fifo.QueueState(T=T, n_chunks=N, step=s_ck, next_id=n_pushed,
+                         entries=[fifo.Entry(head + i, info["levels"][i], lat[i].astype(np.float64))
+                                  for i in range(n_q)],
+                         pred_id=head - 1, pred_kv=[(kv[l, 0], kv[l, 1]) for l in range(m.n_layers)])
+    tr = fifo.queue_step(st, fn, noise[n_pushed])
+    assert tr.popped == [head] and tr.chunk_ids == info["ids"]
+    assert rel_l2(popped, st.ready[0][1]) <= 2e-2
+    for i, e in enumerate(st.entries):
+        assert rel_l2(rest[i], e.latent) <= 2e-2, i
+    for l in range(m.n_layers):
+        assert rel_l2(new_kv[l, 0], st.pred_kv[l][0]) <= 2e-2, l
+        assert rel_l2(new_kv[l, 1], st.pred_kv[l][1]) <= 2e-2, l
+    model.close()
+
+
+def test_load_state_rejects_states_no_stream_reaches():
+    """A state is accepted only if a FIFO stream reaches it; a rejected one
+    leaves the queue unchanged.  A state past its last push is restored closed."""
+    w = synth.WORKLOADS["tiny_fp32"]
+    m, q = w.model, w.queue
+    model, queue, _, _ = make(w, "fp32", n_chunks=-1, T=4)
+    shape = q.chunk_shape(m)
+    Lc = q.tokens_per_chunk(m)
+    kv = np.zeros((m.n_layers, 2, Lc, m.dim), np.float32)
+    queue.step(None)
+    before = queue.inspect()
+    lat2 = np.zeros((2,) + shape, np.float32)
+    from chunked_fifo_denoising_b200 import DPError
+    # head chunk 3 at level 2 while chunk 2 (level 1) has not left
+    with pytest.raises(DPError, match="INVALID_ARG"):
+        queue.load_state(5, 5, lat2, kv)
+    # empty queue at step 3 with 3 chunks pushed: chunks 0..2 are still queued
+    with pytest.raises(DPError, match="INVALID_ARG"):
+        queue.load_state(3, 3, np.zeros((0,) + shape, np.float32))
+    # chunk 2 would be at level 0: it has already left
+    with pytest.raises(DPError, match="INVALID_ARG"):
+        queue.load_state(6, 6, np.zeros((4,) + shape, np.float32), kv)
+    assert queue.inspect() == before
+    # reachable: step 5, chunks 2..4 at levels 1..3, chunk 5 due (open)
+    queue.load_state(5, 5, np.zeros((3,) + shape, np.float32), kv)
+    info = queue.inspect()
+    assert info["ids"] == [2, 3, 4, 5] and info["levels"] == [1, 2, 3, 4] and info["next_push_id"] == 5
+    # past the last push: chunk 4 alone at level 1 at step 7 -> closed, drains in one step
+    queue.load_state(7, 5, np.zeros((1,) + shape, np.float32), kv)
+    info = queue.inspect()
+    assert info["ids"] == [4] and info["levels"] == [1] and info["next_push_id"] == -1
+    queue.step(None)
+    assert queue.try_step(None) == 6          # DP_ERR_DRAINED
+    queue.sync()
+    model.close()
+
+
+def test_host_pop_reports_a_kernel_that_gave_up_a_wait():
+    """After a kernel on the queue's stream gives up a bounded wait (the self
+    test: an mbarrier nothing completes, 2 s), the next host pop returns
+    DP_ERR_KERNEL (the chunk is consumed); the status word is then clear and the
+    next pop returns DP_OK with a chunk that matches the oracle."""
+    w = synth.WORKLOADS["tiny_fp32"]
+    m, q = w.model, w.queue
+    T, N = 1, 3
+    model, queue, p, text = make(w, "fp32", n_chunks=N, T=T, ready=2)
+    noise = [synth.make_noise(m, q, k) for k in range(N)]
+    queue.step(noise[0])
+    queue.step(noise[1])                      # chunks 0 and 1 ready
+    queue.selftest_timeout()
+    out = np.empty(q.chunk_shape(m), np.float32)
+    st, cid = queue.try_pop(out)
+    assert st == 8 and cid == 0               # DP_ERR_KERNEL
+    st, cid = queue.try_pop(out)
+    assert st == 0 and cid == 1
+    fn = dit.make_velocity_fn(p, text, m, T)
+    ready, _ = fifo.run_stream(fn, lambda k: noise[k], T, N)
+    assert rel_l2(out, dict(ready)[1]) <= 1e-4
+    queue.sync()
     model.close()
 
 
