@@ -12,6 +12,7 @@ tensor-core peak reached by the step's algorithmic FLOPs.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload NAME] [--fill steps|load] [--plateau]
                     [--neighbours pred|both] [--qk-norm-rope]
+    python bench.py --stream [--workload wan1.3b_480p_long] [--stream-lengths 32,64]
 
 N > 1 runs N independent replicas (one queue per GPU, no collective on the
 data path), launched by torch.distributed.run.  --impl reference times the
@@ -20,8 +21,13 @@ float64 CPU oracle on a bounded sample of the same step (rank 0 only).
 real steps (needed for the Wan-14B shapes, where a step takes seconds);
 --plateau also times the partial-queue steady state of a stream shorter than
 the queue.  Besides the metric, the line reports the roofline of the GEMM
-class, the per-class kernel times, end-to-end throughput with host buffers,
-clocks sampled during the timed region, device memory and the CPU oracle.
+class, the per-class kernel times (from a separate instrumented pass),
+end-to-end throughput with host buffers (host clock), clocks sampled during
+the timed region, device memory and the CPU oracle.
+--stream runs whole streams instead (every step from the first push to the
+last pop, popping to host), for the workload's own length and the lengths of
+--stream-lengths, and reports the steady-state and whole-stream rates and the
+peak device memory of each, which does not depend on the stream length.
 """
 from __future__ import annotations
 
@@ -267,15 +273,23 @@ def run_reference(args, w):
     vals = []
     t_sample = 0.0
     threads = 1
+    t_start = time.perf_counter()
     for i in range(args.warmup + args.steps):
         v, t_sample, threads = oracle_sample(w)
         if i >= args.warmup:
             vals.append(v)
     v = statistics.median(vals)
+    scale = w.queue.T * w.model.n_layers
     sample = (f"1 chunk x 1 layer of the {w.name} step (with its predecessor K/V), "
-              f"{t_sample:.1f} s each, scaled by T x layers = {w.queue.T * w.model.n_layers}")
+              f"{t_sample:.1f} s each, scaled by T x layers = {scale}")
+    # Each timed "step" is one bounded sample: ms_per_step is the extrapolated
+    # time of a whole step, not the time this run spent per sample.
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": w.queue.frames_per_chunk / v * 1e3,
+            "extrapolated": True,
+            "measured": {"samples": args.steps, "warmup_samples": args.warmup,
+                         "seconds_per_sample": t_sample, "sample_scale_to_step": scale,
+                         "wall_s": time.perf_counter() - t_start},
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": w.name},
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": threads, "kind": "oracle", "sample": sample},
@@ -284,12 +298,9 @@ def run_reference(args, w):
     return 0
 
 
-def run_ours(args, w):
-    import numpy as np
+def setup_rank():
+    """(world, rank, local rank, torch.distributed or None) of this process."""
     import torch
-
-    from chunked_fifo_denoising_b200 import Model, Queue
-
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -300,19 +311,17 @@ def run_ours(args, w):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local))
-    if args.qk_norm_rope:
-        import synth as _s
-        w = _s.with_qk_norm_rope(w)
-    m, q = w.model, w.queue
-    T = q.T
-    occ = T
-    stream = torch.cuda.current_stream()
-    # random-init weights on the device, N(0, 0.02^2), seeded per rank
-    g = torch.Generator(device="cuda").manual_seed(1000 + rank)
+    return world, rank, local, dist
+
+
+def build_model(m, g, stream, neighbours):
+    """The model with random-init weights drawn on the device, N(0, 0.02^2)
+    (RMSNorm weights around 1), and a N(0,1) prompt."""
+    import torch
+
     import synth
-    torch.cuda.synchronize()
-    free0 = torch.cuda.mem_get_info()[0]
-    model = Model(m, "bf16", stream=stream, neighbours=args.neighbours)
+    from chunked_fifo_denoising_b200 import Model
+    model = Model(m, "bf16", stream=stream, neighbours=neighbours)
     for name, shape, per_layer in synth.param_specs(m):
         for l in range(m.n_layers if per_layer else 1):
             t = torch.randn(shape, generator=g, device="cuda") * 0.02
@@ -321,7 +330,27 @@ def run_ours(args, w):
             model.set_param(name, t, l)
             del t
     text = torch.randn((m.text_len, m.text_in_dim), generator=g, device="cuda")
-    n_chunks = T + 1 + args.warmup + args.steps + args.e2e_steps + 2
+    return model, text
+
+
+def run_ours(args, w):
+    import torch
+
+    from chunked_fifo_denoising_b200 import Queue
+
+    world, rank, local, dist = setup_rank()
+    if args.qk_norm_rope:
+        import synth as _s
+        w = _s.with_qk_norm_rope(w)
+    m, q = w.model, w.queue
+    T = q.T
+    occ = T
+    stream = torch.cuda.current_stream()
+    g = torch.Generator(device="cuda").manual_seed(1000 + rank)   # seeded per rank
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    model, text = build_model(m, g, stream, args.neighbours)
+    n_chunks = T + 1 + args.warmup + args.steps + args.kernel_steps + args.e2e_steps + 2
     torch.cuda.synchronize()
     free1 = torch.cuda.mem_get_info()[0]
     queue = Queue(model, text, T, q.frames_per_chunk, q.lat_h, q.lat_w, n_chunks,
@@ -352,8 +381,7 @@ def run_ours(args, w):
         queue.step(None)
         queue.pop(out)
     queue.sync()
-    # timed region: K full steps, per-kernel events on the queue's stream
-    queue.set_timing(True)
+    # timed region: K full steps (no per-kernel instrumentation inside it)
     clocks = Clocks(visible_index(local))
     if dist is not None:
         dist.barrier()
@@ -371,21 +399,36 @@ def run_ours(args, w):
     ck = clocks.stop()
     queue.sync()
     ms = e0.elapsed_time(e1)
+    # per-kernel breakdown from a separate instrumented pass (CUDA events
+    # around every launch on the queue's stream)
+    queue.set_timing(True)
+    torch.cuda.synchronize()
+    k0 = torch.cuda.Event(enable_timing=True)
+    k1 = torch.cuda.Event(enable_timing=True)
+    k0.record(stream)
+    for _ in range(args.kernel_steps):
+        queue.step(None)
+        queue.pop(out)
+    k1.record(stream)
+    torch.cuda.synchronize()
+    ms_instr = k0.elapsed_time(k1)
     kt = queue.timing()
     queue.set_timing(False)
-    # end to end through the public API with host buffers (H2D noise, D2H chunk)
+    queue.sync()
+    # end to end through the public API with page-locked host buffers: every
+    # step copies its noise chunk in (H2D) and the popped chunk out (D2H, the
+    # call returns once it has landed); host clock around the calls
     hn = torch.randn(queue.chunk_shape, generator=torch.Generator().manual_seed(rank)).pin_memory()
     ho = torch.empty(queue.chunk_shape).pin_memory()
     torch.cuda.synchronize()
-    f0 = torch.cuda.Event(enable_timing=True)
-    f1 = torch.cuda.Event(enable_timing=True)
-    f0.record(stream)
+    if dist is not None:
+        dist.barrier()
+    t0 = time.perf_counter()
     for _ in range(args.e2e_steps):
         queue.step(hn)
         queue.pop(ho)
-    f1.record(stream)
     torch.cuda.synchronize()
-    ms_e2e = f0.elapsed_time(f1)
+    ms_e2e = (time.perf_counter() - t0) * 1e3
     queue.sync()
     # max over ranks
     ms, ms_e2e = max_over_ranks([ms, ms_e2e], dist, device="cuda")
@@ -398,7 +441,9 @@ def run_ours(args, w):
     peak_tf = pk["bf16_tflops_sustained"]
     gemm = kt["gemm"]
     attn = kt["self_attention"]
-    launches = sum(v["launches"] for v in kt.values())
+    ks = args.kernel_steps
+    # launches of the library's kernels per step (counted by its per-class timer)
+    launches_per_step = sum(v["launches"] for v in kt.values()) / ks
     roof = {"bound": "tensor", "kernel": "gemm_tc (tcgen05 GEMM, all fused epilogues)",
             "achieved": gemm["flops"] / (gemm["ms"] / 1e3) / 1e12 if gemm["ms"] > 0 else None,
             "peak": peak_tf, "unit": "TFLOP/s",
@@ -421,13 +466,16 @@ def run_ours(args, w):
             "pct_bf16_peak": 100.0 * flops / (ms_step / 1e3) / (peak_tf * 1e12),
             "step_tflop": flops / 1e12,
             "roofline": roof,
-            "kernels": {k: {"ms_per_step": v["ms"] / args.steps, "launches_per_step": v["launches"] / args.steps,
+            "kernels": {k: {"ms_per_step": v["ms"] / ks, "launches_per_step": v["launches"] / ks,
                             "tflops": (v["flops"] / (v["ms"] / 1e3) / 1e12) if v["ms"] > 0 and v["flops"] else None,
                             "gbs": (v["bytes"] / (v["ms"] / 1e3) / 1e9) if v["ms"] > 0 and v["bytes"] else None}
                         for k, v in kt.items() if v["launches"]},
+            "kernels_pass": {"steps": ks, "ms_per_step_instrumented": ms_instr / ks,
+                             "note": "separate pass after the timed region, CUDA events around every launch"},
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(hn.numel() * 4),
-                    "d2h_bytes_per_step": int(ho.numel() * 4), "steps": args.e2e_steps},
-            "gpu_launches": launches, "clocks": ck,
+                    "d2h_bytes_per_step": int(ho.numel() * 4), "steps": args.e2e_steps,
+                    "clock": "host perf_counter around dp_queue_step(host noise) + dp_queue_pop(host out)"},
+            "gpu_launches": int(round(launches_per_step * args.steps)), "clocks": ck,
             "memory": {"model_bytes": int(free0 - free1), "queue_bytes": int(free1 - free2),
                        "source": "cudaMemGetInfo around dp_model_create+set_param and dp_queue_init"},
             "fill": args.fill}
@@ -461,12 +509,112 @@ def run_ours(args, w):
     return 0
 
 
+def stream_summary(step_ms, occupancy, T, frames, wall_s, n_chunks):
+    """Rates of one whole stream: steady state (steps with all T levels
+    occupied: one chunk leaves per step) and whole stream (every chunk's frames
+    over the host wall time from the first push to the last pop)."""
+    steady = [t for t, n in zip(step_ms, occupancy) if n == T]
+    out = {"chunks": n_chunks, "steps": len(step_ms), "wall_s": wall_s,
+           "frames": n_chunks * frames, "whole_stream_frames_per_s": n_chunks * frames / wall_s,
+           "steady_steps": len(steady)}
+    if steady:
+        med = statistics.median(steady)
+        out["steady_ms_per_step"] = med
+        out["steady_frames_per_s"] = frames / (med / 1e3)
+    return out
+
+
+def run_stream(args, w):
+    """Whole streams of the workload's model, from the first push to the last
+    pop (fill, steady state, drain), one per stream length, on one queue each:
+    host pops every clean chunk to page-locked memory, device memory is sampled
+    after every step.  The longest stream's steady state is the line's value."""
+    import torch
+
+    from chunked_fifo_denoising_b200 import Queue
+
+    world, rank, local, dist = setup_rank()
+    m, q = w.model, w.queue
+    T, frames = q.T, q.frames_per_chunk
+    stream = torch.cuda.current_stream()
+    g = torch.Generator(device="cuda").manual_seed(1000 + rank)
+    model, text = build_model(m, g, stream, args.neighbours)
+    total = torch.cuda.mem_get_info()[1]
+    lengths = sorted(set([int(x) for x in args.stream_lengths.split(",") if x] + [q.n_chunks]))
+    runs = []
+    clocks = Clocks(visible_index(local))
+    for n in lengths:
+        torch.cuda.synchronize()
+        free0 = torch.cuda.mem_get_info()[0]
+        queue = Queue(model, text, T, frames, q.lat_h, q.lat_w, n, ready_capacity=2, seed=3 + rank)
+        torch.cuda.synchronize()
+        free1 = torch.cuda.mem_get_info()[0]
+        peak_used = total - free1
+        ho = torch.empty(queue.chunk_shape).pin_memory()
+        step_ms, occupancy, popped = [], [], []
+        if dist is not None:
+            dist.barrier()
+        t0 = time.perf_counter()
+        while True:
+            info = queue.inspect()
+            if info["drained"]:
+                break
+            ts = time.perf_counter()
+            queue.step(None)
+            while True:
+                st, cid = queue.try_pop(ho)
+                if st != 0:
+                    break
+                popped.append(cid)
+            queue.sync()
+            step_ms.append((time.perf_counter() - ts) * 1e3)
+            occupancy.append(info["n"])
+            peak_used = max(peak_used, total - torch.cuda.mem_get_info()[0])
+        wall = time.perf_counter() - t0
+        assert popped == list(range(n)), "chunks must pop in push order"
+        r = stream_summary(step_ms, occupancy, T, frames, wall, n)
+        r.update({"queue_bytes": int(free0 - free1), "peak_device_bytes_used": int(peak_used)})
+        runs.append(r)
+        queue.close()
+    ck = clocks.stop()
+    head = runs[-1]
+    peaks_equal = len({r["peak_device_bytes_used"] for r in runs}) == 1
+    vals = max_over_ranks([head["wall_s"], head.get("steady_ms_per_step", 0.0)], dist, device="cuda")
+    line = {"metric": METRIC, "mode": "stream",
+            "value": world * frames / (vals[1] / 1e3) if vals[1] > 0 else None, "unit": UNIT,
+            "n_gpus": world, "steps": head["steps"], "warmup": 0,
+            "ms_per_step": vals[1], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic: seeded N(0,1) noise per chunk (device generator), "
+                                     "N(0,1) prompt, N(0,0.02^2) random-init weights",
+            "config": {"workload": w.name, "T": T, "chunks": q.n_chunks, "frames_per_chunk": frames,
+                       "layers": m.n_layers, "dim": m.dim, "chunk_tokens": q.tokens_per_chunk(m),
+                       "parallelism": f"replicas x{world}"},
+            "whole_stream_frames_per_s": world * head["frames"] / vals[0],
+            "streams": runs,
+            "memory_flat_in_stream_length": peaks_equal,
+            "memory_source": "cudaMemGetInfo (device-wide bytes in use) after dp_queue_init and after every step",
+            "clocks": ck}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    model.close()
+    if dist is not None:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--kernel-steps", type=int, default=2,
+                    help="steps of the separate per-kernel timing pass")
+    ap.add_argument("--stream", action="store_true",
+                    help="run whole streams (fill, steady state, drain) instead of timing the "
+                         "steady state alone; reports stream rates and peak device memory")
+    ap.add_argument("--stream-lengths", default="32,64",
+                    help="stream lengths (chunks) run besides the workload's own, with --stream")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="wan1.3b_480p")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -487,6 +635,8 @@ def main():
     w = synth.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.stream:
+        return run_stream(args, w)
     return run_ours(args, w)
 
 

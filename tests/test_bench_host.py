@@ -82,3 +82,25 @@ def test_peaks_come_from_the_measured_file():
     pk = bench.peaks()
     assert pk["_source"] in ("measured", "fallback")
     assert pk["bf16_tflops_sustained"] > 0 and pk["hbm_gbs"] > 0
+
+
+def test_stream_summary_rates():
+    """Whole stream: N chunks x F frames over the wall time; steady state: the
+    median step with all T levels occupied (one chunk leaves per step)."""
+    T, F = 3, 2
+    occ = [1, 2, 3, 3, 3, 2, 1]          # N = 5 chunks, N + T - 1 = 7 steps
+    ms = [100.0, 200.0, 300.0, 310.0, 290.0, 200.0, 100.0]
+    r = bench.stream_summary(ms, occ, T, F, wall_s=1.6, n_chunks=5)
+    assert r["steps"] == 7 and r["steady_steps"] == 3
+    assert r["steady_ms_per_step"] == 300.0
+    assert r["steady_frames_per_s"] == pytest.approx(F / 0.3)
+    assert r["whole_stream_frames_per_s"] == pytest.approx(10 / 1.6)
+
+
+def test_long_stream_schedule_is_177_steps():
+    """128 chunks through a T = 50 queue: 128 + 50 - 1 = 177 steps, 79 of them
+    with all 50 levels occupied."""
+    w = synth.WORKLOADS["wan1.3b_480p_long"]
+    N, T = w.queue.n_chunks, w.queue.T
+    occ = [min(s, N - 1) - max(0, s - T + 1) + 1 for s in range(N + T - 1)]
+    assert len(occ) == 177 and occ.count(T) == N - T + 1 == 79
