@@ -27,13 +27,15 @@ The pages give no formula for the DiT block, the timestep embedding or the
 flow parameterisation.  Every step they leave open is written here in its
 plainest form and marked ``reading:`` at the point of use.
 
-Parity status: the self-attention, softmax, layer norm, modulation, GELU, SiLU,
-sinusoid, patch (un)folding, Euler update and queue bookkeeping are pinned by
-tests that do not reuse this code (closed forms, brute-force loops, textbook
-values, invariants and a hand-derived queue trace).  The composition of these
-pieces into the full DiT velocity has no printed value on the pages to pin it
-against: "parity unpinned" for ``dit.velocity`` beyond the invariants the tests
-check (gates, causality of the predecessor link, batch independence).
+Parity status: every function here is pinned by tests that do not reuse this
+code (tests/test_oracle_pins.py, tests/test_oracle_composition_pins.py):
+closed forms, brute-force loops, textbook values, invariants, a hand-derived
+queue trace, and hand-derived values (fixtures under tests/golden/) for the
+per-level timestep embedding and modulation, the prompt's per-layer K/V and
+the composed DiT velocity of a one-layer d = 4 model on two chunks.  Planted
+mistakes (a swapped shift and scale, a misordered modulation split, swapped
+gates, a missing SiLU, an unscaled timestep, the tanh GELU, a dropped LN eps)
+each break one of them.
 """
 
 from . import dit, fifo  # noqa: F401
