@@ -104,6 +104,27 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// P = 2^(S * sl2 - m) of one thread's 128-key row of S (MUFU ex2), written
+// back over S in TMEM as bf16 pairs; the fp32 values are summed into four
+// packed partial sums.
+__device__ __forceinline__ void exp_tile(const float (&s)[128], uint64_t sl2x2, uint64_t nmx2, uint32_t tS,
+                                         uint64_t (&sp2)[4]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float xa, xb;
+      f2_unpack(f2_fma(f2_pack(s[32 * q + 2 * i], s[32 * q + 2 * i + 1]), sl2x2, nmx2), xa, xb);
+      const float a = ex2_approx(xa);
+      const float b = ex2_approx(xb);
+      sp2[i & 3] = f2_add(sp2[i & 3], f2_pack(a, b));
+      w[i] = pack_bf16(a, b);
+    }
+    tmem_st16_nowait(tS + q * 16, w);
+  }
+}
+
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const unsigned long long t0 = globaltimer();
   while (!mbar_try_wait(bar, parity)) {
@@ -270,17 +291,26 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
       uint32_t gk = 0;          // K/V tiles consumed so far
       uint32_t gp[2] = {0, 0};  // P tiles of tile A / tile B consumed so far
       bool ok = true;
+      // The first S of a block is issued at the end of the previous block,
+      // right after that block's last PV of tile A, so the tensor core has work
+      // while the softmax warps finish the last tile (several blocks per CTA).
+      bool first_issued = false;
       for (int qb = qb0; qb < qb1 && ok; ++qb) {
         const int bi = qb - qb0;
         const bool has_b = qb * 2 * BQ + BQ < p.Lq;
-        ok = mbar_wait(&q_full, bi & 1, &abort_flag, status, ST_TIMEOUT_ATTN) &&
-             mbar_wait(&k_full[gk & 1], (gk >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN);
-        if (!ok) break;
-        tc_fence_after();
-        issue_s(0, gk);
-        if (has_b) issue_s(1, gk);
-        mma_commit(&k_empty[gk & 1]);
-        if (nt == 1) mma_commit(&q_empty);  // last S of this block issued
+        if (!first_issued) {
+          ok = mbar_wait(&q_full, bi & 1, &abort_flag, status, ST_TIMEOUT_ATTN) &&
+               mbar_wait(&k_full[gk & 1], (gk >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(0, gk);
+          if (has_b) issue_s(1, gk);
+          mma_commit(&k_empty[gk & 1]);
+          if (nt == 1) mma_commit(&q_empty);  // last S of this block issued
+        }
+        first_issued = false;
+        const bool more = qb + 1 < qb1;
+        const bool next_has_b = (qb + 1) * 2 * BQ + BQ < p.Lq;
         for (int j = 0; j < nt; ++j) {
           const uint32_t g = gk + j;
           const bool next = j + 1 < nt;
@@ -294,6 +324,16 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
           ++gp[0];
           if (next) {
             if (!mbar_wait(&k_full[(g + 1) & 1], ((g + 1) >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(0, g + 1);
+          } else if (more) {
+            // the next block's Q (loaded once this block's last S was issued)
+            // and its first key tile
+            if (!mbar_wait(&q_full, (bi + 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN) ||
+                !mbar_wait(&k_full[(g + 1) & 1], ((g + 1) >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) {
               ok = false;
               break;
             }
@@ -314,6 +354,11 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
             if (has_b) issue_s(1, g + 1);
             mma_commit(&k_empty[(g + 1) & 1]);
             if (j + 2 == nt) mma_commit(&q_empty);  // last S of this block issued
+          } else if (more) {
+            if (next_has_b) issue_s(1, g + 1);
+            mma_commit(&k_empty[(g + 1) & 1]);
+            if (nt == 1) mma_commit(&q_empty);    // last S of the next block issued
+            first_issued = true;
           }
         }
         gk += nt;
@@ -369,20 +414,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
         // P (bf16, two keys per 32-bit column) over the first 64 columns of S, 32
         // keys at a time; S is already in registers, and PV of the previous tile
         // (which read the old P) completed before S of this tile was written
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t w[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float xa, xb;
-            f2_unpack(f2_fma(f2_pack(s[32 * q + 2 * i], s[32 * q + 2 * i + 1]), sl2x2, nmx2), xa, xb);
-            const float a = ex2_approx(xa);
-            const float b = ex2_approx(xb);
-            sp2[i & 3] = f2_add(sp2[i & 3], f2_pack(a, b));
-            w[i] = pack_bf16(a, b);
-          }
-          tmem_st16_nowait(tS + q * 16, w);
-        }
+        exp_tile(s, sl2x2, nmx2, tS, sp2);
         tmem_wait_st();
         if (resc && j > 0) {
           // O must hold PV of every earlier tile of this block before it is rescaled

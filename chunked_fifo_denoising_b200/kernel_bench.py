@@ -21,6 +21,8 @@ CASES = {
     # name: (kind, dict)
     "qkv": ("gemm", dict(N=4608, K=1536, epi=B.DP_EPI_STORE)),
     "oproj": ("gemm", dict(N=1536, K=1536, epi=B.DP_EPI_RESID_GATED)),
+    "crossq": ("gemm", dict(N=1536, K=1536, epi=B.DP_EPI_STORE)),
+    "crosso": ("gemm", dict(N=1536, K=1536, epi=B.DP_EPI_RESID)),
     "ffn1": ("gemm", dict(N=8960, K=1536, epi=B.DP_EPI_GELU)),
     "ffn2": ("gemm", dict(N=1536, K=8960, epi=B.DP_EPI_RESID_GATED)),
     "ffn1_14b": ("gemm", dict(N=13824, K=5120, epi=B.DP_EPI_GELU, Lc=7200)),
