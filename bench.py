@@ -72,7 +72,7 @@ def gemm_traffic():
         with open(os.path.join(src, f), "rb") as fh:
             h.update(fh.read())
     try:
-        with open(os.path.join(ROOT, "profiles", "step_launches_wan1.3b.md")) as fh:
+        with open(os.path.join(ROOT, "profiles", "gemm_traffic_wan1.3b.md")) as fh:
             text = fh.read()
     except OSError:
         return None
@@ -448,7 +448,8 @@ def run_ours(args, w):
             "achieved": gemm["flops"] / (gemm["ms"] / 1e3) / 1e12 if gemm["ms"] > 0 else None,
             "peak": peak_tf, "unit": "TFLOP/s",
             "peak_source": f"{pk['_source']} bf16_tflops_sustained (kernel timed inside a long step)",
-            "traffic": gemm_traffic(), "traffic_unit": "bytes per launch (ncu, one step's launches averaged)"}
+            "traffic": gemm_traffic(),
+            "traffic_unit": "bytes per launch (ncu, small per-kernel captures scaled to full size; mean of the six GEMM shapes)"}
     if roof["achieved"]:
         roof["frac"] = roof["achieved"] / peak_tf
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -67,7 +67,7 @@ def test_gemm_traffic_follows_the_kernel_source():
     for f in ("k_gemm_tc.cu", "tc_common.cuh"):
         with open(os.path.join(src, f), "rb") as fh:
             h.update(fh.read())
-    with open(os.path.join(ROOT, "profiles", "step_launches_wan1.3b.md")) as fh:
+    with open(os.path.join(ROOT, "profiles", "gemm_traffic_wan1.3b.md")) as fh:
         text = fh.read()
     line = [l for l in text.splitlines() if l.startswith("traffic gemm_tc_kernel")]
     assert len(line) == 1
