@@ -57,6 +57,8 @@ struct AttnParams {
   void* out; long long ldo;
   int succ_in_batch;              // chunk c < n_chunks-1 also reads chunk c+1's own keys
   int qblocks_per_cta;            // tensor-core path: 256-query blocks per CTA (0 = choose)
+  int dual_rem;                   // tensor-core path, set by the launcher: the last grid
+                                  // column pairs two heads' one-tile remainder blocks
 };
 
 struct LnParams {

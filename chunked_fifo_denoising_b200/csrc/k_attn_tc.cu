@@ -12,7 +12,10 @@
 //
 // CTA = 256-query blocks (two 128-row tiles A and B each) of one (chunk, head),
 // processed one after the other with TMEM and barriers kept (several blocks
-// per CTA when the key set is short), 10 warps:
+// per CTA when the key set is short).  With a long key set, a chunk whose last
+// block holds one tile of rows (3120 = 12 x 256 + 48) has the last blocks of
+// heads h and h + 1 paired in one CTA as its tiles A and B, each with its own
+// head's K/V.  10 warps:
 //   warp 0      TMA producer: Q_A, Q_B once; K and V tiles of 128 keys into two
 //               2-stage rings, each tile from whichever buffer it belongs to
 //   warp 1      TMEM owner + MMA issuer, tiles ping-ponged on the tensor core:
@@ -145,10 +148,17 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y, c = blockIdx.z;
-  // this CTA covers 256-query blocks [qb0, qb1) of chunk c, one after the other
   const int nqb = (p.Lq + 2 * BQ - 1) / (2 * BQ);
-  const int qb0 = blockIdx.x * p.qblocks_per_cta;
-  const int qb1 = min(nqb, qb0 + p.qblocks_per_cta);
+  // When the last 256-query block of a chunk holds at most 128 rows (one
+  // tile), the last grid column pairs the last blocks of heads h and h + 1
+  // (h even) as tiles A and B: each tile reads its own head's K/V, one ring
+  // slot per head, and the column of odd h has nothing to do.  The other
+  // columns cover blocks [qb0, qb1) of head h, one after the other.
+  const bool dual = p.dual_rem && blockIdx.x == gridDim.x - 1;
+  if (dual && (h & 1)) return;
+  const int hB = dual ? h + 1 : h;  // head of tile B
+  const int qb0 = dual ? nqb - 1 : blockIdx.x * p.qblocks_per_cta;
+  const int qb1 = dual ? nqb : min(nqb - (p.dual_rem ? 1 : 0), qb0 + p.qblocks_per_cta);
   // key sources of this chunk (the same for every query block)
   int n_p = 0;
   bool pred_cache = false;
@@ -192,27 +202,30 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
   if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
-      const int col0 = h * HD;
+      const int col0 = h * HD, colB = hB * HD;
       uint32_t issued_k = 0, issued_v = 0, par = 0, q_issued = 0;
-      uint32_t gk = 0;  // K/V tiles issued so far (stage gk & 1, use gk >> 1)
+      // K/V tiles issued so far: a two-stage ring (stage gk & 1, use gk >> 1);
+      // paired heads: one stage holding both heads' tiles (use gk)
+      uint32_t gk = 0;
       bool ok = true;
       for (int qb = qb0; qb < qb1 && ok; ++qb) {
         const int bi = qb - qb0;
         const int q0 = qb * 2 * BQ;
-        const bool has_b = q0 + BQ < p.Lq;
+        const bool has_b = dual || q0 + BQ < p.Lq;
         const int qrow0 = c * p.Lq + q0;
+        const int qrowB = dual ? qrow0 : qrow0 + BQ;
         // Q of the previous block is read by its S MMAs only
         if (bi > 0 && !mbar_wait(&q_empty, (bi - 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) break;
         mbar_arrive_expect_tx(&q_full, (has_b ? 2 : 1) * C::T_BYTES);
 #pragma unroll
         for (int s = 0; s < C::NSUB; ++s) {
           tma_load_2d(smem + C::OFF_QA + s * C::SUB_BYTES, &maps.q, col0 + 64 * s, qrow0, &q_full);
-          if (has_b) tma_load_2d(smem + C::OFF_QB + s * C::SUB_BYTES, &maps.q, col0 + 64 * s, qrow0 + BQ, &q_full);
+          if (has_b) tma_load_2d(smem + C::OFF_QB + s * C::SUB_BYTES, &maps.q, colB + 64 * s, qrowB, &q_full);
         }
         q_issued = bi + 1;
         for (int j = 0; j < nt; ++j, ++gk) {
-          const int st = gk & 1;
-          const uint32_t use = gk >> 1;
+          const int st = dual ? 0 : (int)(gk & 1);
+          const uint32_t use = dual ? gk : gk >> 1;
           const CUtensorMap* mk;
           const CUtensorMap* mv;
           int row;
@@ -239,20 +252,24 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&k_full[st], C::T_BYTES);
+          mbar_arrive_expect_tx(&k_full[st], (dual ? 2 : 1) * C::T_BYTES);
 #pragma unroll
-          for (int s = 0; s < C::NSUB; ++s)
+          for (int s = 0; s < C::NSUB; ++s) {
             tma_load_2d(smem + C::OFF_K + st * C::T_BYTES + s * C::SUB_BYTES, mk, col0 + 64 * s, row, &k_full[st]);
+            if (dual) tma_load_2d(smem + C::OFF_K + C::T_BYTES + s * C::SUB_BYTES, mk, colB + 64 * s, row, &k_full[st]);
+          }
           issued_k |= 1u << st;
           par = (par & ~(1u << st)) | ((use & 1u) << st);
           if (use > 0 && !mbar_wait(&v_empty[st], (use - 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&v_full[st], C::T_BYTES);
+          mbar_arrive_expect_tx(&v_full[st], (dual ? 2 : 1) * C::T_BYTES);
 #pragma unroll
-          for (int s = 0; s < C::NSUB; ++s)
+          for (int s = 0; s < C::NSUB; ++s) {
             tma_load_2d(smem + C::OFF_V + st * C::T_BYTES + s * C::SUB_BYTES, mv, col0 + 64 * s, row, &v_full[st]);
+            if (dual) tma_load_2d(smem + C::OFF_V + C::T_BYTES + s * C::SUB_BYTES, mv, colB + 64 * s, row, &v_full[st]);
+          }
           issued_v |= 1u << st;
         }
       }
@@ -269,9 +286,14 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
       // ---------------- MMA issuer ----------------
       constexpr uint32_t IDESC_S = idesc_bf16_f32(BQ, BKV, 0, 0);
       constexpr uint32_t IDESC_O = idesc_bf16_f32(BQ, HD, 0, 1);
+      // ring stage and phase of K/V tile g; with paired heads one stage holds
+      // both heads' tiles (slot X) and its phase flips every tile
+      auto kv_st = [&](uint32_t g) -> int { return dual ? 0 : (int)(g & 1); };
+      auto kv_par = [&](uint32_t g) -> uint32_t { return dual ? (g & 1) : ((g >> 1) & 1); };
+      auto kv_slot = [&](int X, uint32_t g) -> uint32_t { return dual ? (uint32_t)X : (g & 1); };
       auto issue_s = [&](int X, uint32_t g) {
         const uint32_t sQ = smem_u32(smem + (X ? C::OFF_QB : C::OFF_QA));
-        const uint32_t sK = smem_u32(smem + C::OFF_K + (g & 1) * C::T_BYTES);
+        const uint32_t sK = smem_u32(smem + C::OFF_K + kv_slot(X, g) * C::T_BYTES);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::SUB_BYTES + (kk & 3) * 32;
@@ -281,7 +303,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
         mma_commit(&s_full[X]);
       };
       auto issue_pv = [&](int X, uint32_t g, int j) {
-        const uint32_t sV = smem_u32(smem + C::OFF_V + (g & 1) * C::T_BYTES);
+        const uint32_t sV = smem_u32(smem + C::OFF_V + kv_slot(X, g) * C::T_BYTES);
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk)  // 16 keys = 8 TMEM columns of packed P; 2 atoms of V
           mma_bf16_ts(tmem + C::o_col(X), tmem + C::s_col(X) + kk * 8,
@@ -297,15 +319,15 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
       bool first_issued = false;
       for (int qb = qb0; qb < qb1 && ok; ++qb) {
         const int bi = qb - qb0;
-        const bool has_b = qb * 2 * BQ + BQ < p.Lq;
+        const bool has_b = dual || qb * 2 * BQ + BQ < p.Lq;
         if (!first_issued) {
           ok = mbar_wait(&q_full, bi & 1, &abort_flag, status, ST_TIMEOUT_ATTN) &&
-               mbar_wait(&k_full[gk & 1], (gk >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN);
+               mbar_wait(&k_full[kv_st(gk)], kv_par(gk), &abort_flag, status, ST_TIMEOUT_ATTN);
           if (!ok) break;
           tc_fence_after();
           issue_s(0, gk);
           if (has_b) issue_s(1, gk);
-          mma_commit(&k_empty[gk & 1]);
+          mma_commit(&k_empty[kv_st(gk)]);
           if (nt == 1) mma_commit(&q_empty);  // last S of this block issued
         }
         first_issued = false;
@@ -314,7 +336,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
         for (int j = 0; j < nt; ++j) {
           const uint32_t g = gk + j;
           const bool next = j + 1 < nt;
-          if (!mbar_wait(&v_full[g & 1], (g >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN) ||
+          if (!mbar_wait(&v_full[kv_st(g)], kv_par(g), &abort_flag, status, ST_TIMEOUT_ATTN) ||
               !mbar_wait(&p_full[0], gp[0] & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) {
             ok = false;
             break;
@@ -323,7 +345,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
           issue_pv(0, g, j);
           ++gp[0];
           if (next) {
-            if (!mbar_wait(&k_full[(g + 1) & 1], ((g + 1) >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) {
+            if (!mbar_wait(&k_full[kv_st(g + 1)], kv_par(g + 1), &abort_flag, status, ST_TIMEOUT_ATTN)) {
               ok = false;
               break;
             }
@@ -333,7 +355,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
             // the next block's Q (loaded once this block's last S was issued)
             // and its first key tile
             if (!mbar_wait(&q_full, (bi + 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN) ||
-                !mbar_wait(&k_full[(g + 1) & 1], ((g + 1) >> 1) & 1, &abort_flag, status, ST_TIMEOUT_ATTN)) {
+                !mbar_wait(&k_full[kv_st(g + 1)], kv_par(g + 1), &abort_flag, status, ST_TIMEOUT_ATTN)) {
               ok = false;
               break;
             }
@@ -349,14 +371,14 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
             issue_pv(1, g, j);
             ++gp[1];
           }
-          mma_commit(&v_empty[g & 1]);
+          mma_commit(&v_empty[kv_st(g)]);
           if (next) {
             if (has_b) issue_s(1, g + 1);
-            mma_commit(&k_empty[(g + 1) & 1]);
+            mma_commit(&k_empty[kv_st(g + 1)]);
             if (j + 2 == nt) mma_commit(&q_empty);  // last S of this block issued
           } else if (more) {
             if (next_has_b) issue_s(1, g + 1);
-            mma_commit(&k_empty[(g + 1) & 1]);
+            mma_commit(&k_empty[kv_st(g + 1)]);
             if (nt == 1) mma_commit(&q_empty);    // last S of the next block issued
             first_issued = true;
           }
@@ -380,7 +402,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
     bool ok = true;
     for (int qb = qb0; qb < qb1 && ok; ++qb) {
       const int q0 = qb * 2 * BQ;
-      if (X == 1 && !(q0 + BQ < p.Lq)) continue;  // this block has no tile B
+      if (X == 1 && !dual && !(q0 + BQ < p.Lq)) continue;  // this block has no tile B
       const int qrow0 = c * p.Lq + q0;
       float m = -INFINITY, l = 0.0f;
       for (int j = 0; j < nt; ++j, ++gx) {
@@ -444,8 +466,10 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
       if (!warp_wait(&pv_done[X], (gx - 1) & 1, &abort_flag, status)) { ok = false; break; }
       tc_fence_after();
       const float inv = 1.0f / l;
-      const bool row_ok = q0 + X * BQ + r < p.Lq;
-      bf16* O = (bf16*)p.out + (long long)(qrow0 + X * BQ + r) * p.ldo + h * HD;
+      // tile B holds the next query rows, or (paired heads) the same rows of head hB
+      const int roff = dual ? 0 : X * BQ;
+      const bool row_ok = q0 + roff + r < p.Lq;
+      bf16* O = (bf16*)p.out + (long long)(qrow0 + roff + r) * p.ldo + (X ? hB : h) * HD;
 #pragma unroll 1
       for (int i = 0; i < HD / 32; ++i) {
         float t[32];
@@ -506,7 +530,15 @@ cudaError_t launch(const AttnParams& p, int* status, cudaStream_t s) {
   AttnParams q = p;
   q.qblocks_per_cta = p.qblocks_per_cta > 0 ? p.qblocks_per_cta : (keys <= 1024 ? 4 : 1);
   const int nqb = (p.Lq + 2 * BQ - 1) / (2 * BQ);
-  dim3 grid((nqb + q.qblocks_per_cta - 1) / q.qblocks_per_cta, p.n_heads, p.n_chunks);
+  // A last block of one tile (Lq mod 256 in 1..128) costs a full block's
+  // time for at most half its rows: pair the heads' last blocks in one column.
+  // Only for long key sets (one block per CTA, self-attention): a paired block
+  // has one K/V ring stage per head, which a short key set cannot hide
+  // (cross-attention with 512 keys measured 6 % slower paired).
+  const int last_rows = p.Lq - (nqb - 1) * 2 * BQ;
+  q.dual_rem = (last_rows <= BQ && p.n_heads % 2 == 0 && q.qblocks_per_cta == 1) ? 1 : 0;
+  const int main_blocks = nqb - q.dual_rem;
+  dim3 grid((main_blocks + q.qblocks_per_cta - 1) / q.qblocks_per_cta + q.dual_rem, p.n_heads, p.n_chunks);
   if (!status) status = op_status_word();
   attn_tc_kernel<HD><<<grid, 320, C::SMEM, s>>>(maps, q, status);
   return cudaGetLastError();

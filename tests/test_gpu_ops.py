@@ -202,11 +202,15 @@ def oracle_self_attention(q, k, v, n, Lc, H, kp, vp, rows=None, succ=False):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("hd,Lc,n,cached,succ", [(64, 200, 3, True, False), (128, 333, 2, False, False),
-                                                 (128, 130, 4, True, False), (128, 200, 3, True, True),
-                                                 (64, 333, 2, False, True)])
-def test_self_attention_neighbour_buffers(dtype, hd, Lc, n, cached, succ):
-    H = 2
+@pytest.mark.parametrize("hd,Lc,n,cached,succ,H", [(64, 200, 3, True, False, 2), (128, 333, 2, False, False, 2),
+                                                   (128, 130, 4, True, False, 2), (128, 200, 3, True, True, 2),
+                                                   (64, 333, 2, False, True, 2), (128, 100, 3, True, False, 2),
+                                                   (64, 300, 2, True, True, 3)])
+def test_self_attention_neighbour_buffers(dtype, hd, Lc, n, cached, succ, H):
+    """Ragged chunks: the last 256-query block of a chunk holds Lc mod 256
+    rows; with one tile's worth (333, 100, 300 rows) and an even head count the
+    tensor-core path pairs two heads' last blocks in one CTA (H = 3 keeps them
+    apart)."""
     d = H * hd
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     qkv = gen((n * Lc, 3 * d), 1.0, tdt, seed=30)
@@ -222,8 +226,11 @@ def test_self_attention_neighbour_buffers(dtype, hd, Lc, n, cached, succ):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-def test_cross_attention_shared_keys(dtype):
-    H, hd, Lq, n, Lt = 4, 64, 257, 3, 64
+@pytest.mark.parametrize("Lq", [257, 700])
+def test_cross_attention_shared_keys(dtype, Lq):
+    """Several 256-query blocks per CTA (short key set); Lq = 257 ends in a
+    one-tile block of 1 row, Lq = 700 in a block of two tiles (188 rows)."""
+    H, hd, n, Lt = 4, 64, 3, 64
     d = H * hd
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     q = gen((n * Lq, d), 1.0, tdt, seed=32)
@@ -244,7 +251,7 @@ def test_self_attention_full_size_sampled_rows(succ):
     q, k, v = qkv[:, :d], qkv[:, d:2 * d], qkv[:, 2 * d:]
     cache = gen((Lc, 2 * d), 1.0, torch.bfloat16, seed=41)
     out = run_attn(q, k, v, n, Lc, H, hd, Lc, Lc, 1, cache[:, :d], cache[:, d:], succ=int(succ))
-    rows = np.array([0, 1, 127, 128, 1000, 3119])
+    rows = np.array([0, 1, 127, 128, 1000, 3071, 3072, 3100, 3119])   # 3072..: the paired last block
     qf, kf, vf = f64(q), f64(k), f64(v)
     for c in (0, 1, 17, 49):
         sl = slice(c * Lc, (c + 1) * Lc)
