@@ -52,7 +52,8 @@ struct Cfg {
   static constexpr uint32_t OFF_QB = T_BYTES;
   static constexpr uint32_t OFF_K = 2 * T_BYTES;             // 2 stages
   static constexpr uint32_t OFF_V = OFF_K + 2 * T_BYTES;     // 2 stages
-  static constexpr uint32_t SMEM = OFF_V + 2 * T_BYTES + 1024;
+  static constexpr uint32_t OFF_STG = OFF_V + 2 * T_BYTES;   // 8 x 4 KB output staging boxes
+  static constexpr uint32_t SMEM = OFF_STG + 8 * 4096 + 1024;
   static constexpr uint32_t TMEM_COLS = 512;
   __device__ static constexpr uint32_t s_col(int X) { return X ? 128u : 0u; }
   __device__ static constexpr uint32_t o_col(int X) { return 256u + (X ? (uint32_t)HD : 0u); }
@@ -60,7 +61,26 @@ struct Cfg {
 
 struct AttnMaps {
   CUtensorMap q, k, v, kp, vp;
+  CUtensorMap o;  // output as [chunk][row < Lq][column]: boxes clip at the end of each chunk
 };
+
+// One row of 64 bf16 (128 bytes, in 32 words) into a 32-row box with the
+// 128-byte swizzle of the output tensor map.
+__device__ __forceinline__ void stage_row(uint8_t* box, int r, const uint32_t (&w)[32]) {
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    *reinterpret_cast<uint4*>(box + r * 128 + ((j ^ (r & 7)) << 4)) =
+        make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+}
+
+// 3-D tiled TMA store shared -> global (bulk-group completion).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, int x, int y, int z, const void* smem_src) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(x), "r"(y), "r"(z), "r"(smem_u32(smem_src))
+      : "memory");
+}
 
 // Key tiles of a chunk: predecessor [0, tp), own [tp, tp+to), successor after.
 __device__ __forceinline__ int tile_valid(int j, int tp, int n_p, int to, int n_o, int n_s) {
@@ -291,23 +311,25 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
       auto kv_st = [&](uint32_t g) -> int { return dual ? 0 : (int)(g & 1); };
       auto kv_par = [&](uint32_t g) -> uint32_t { return dual ? (g & 1) : ((g >> 1) & 1); };
       auto kv_slot = [&](int X, uint32_t g) -> uint32_t { return dual ? (uint32_t)X : (g & 1); };
+      // descriptors are built once per operand tile; a K step of 16 columns
+      // adds 32 bytes (2 in the 16-byte address field), a 64-column sub-tile
+      // SUB_BYTES, 16 rows of V 2048 bytes (the field stays below 2^14)
       auto issue_s = [&](int X, uint32_t g) {
-        const uint32_t sQ = smem_u32(smem + (X ? C::OFF_QB : C::OFF_QA));
-        const uint32_t sK = smem_u32(smem + C::OFF_K + kv_slot(X, g) * C::T_BYTES);
+        const uint64_t dq = desc_sw128(smem_u32(smem + (X ? C::OFF_QB : C::OFF_QA)), 16, 1024);
+        const uint64_t dk = desc_sw128(smem_u32(smem + C::OFF_K + kv_slot(X, g) * C::T_BYTES), 16, 1024);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::SUB_BYTES + (kk & 3) * 32;
-          mma_bf16_ss(tmem + C::s_col(X), desc_sw128(sQ + off, 16, 1024), desc_sw128(sK + off, 16, 1024),
-                      IDESC_S, kk > 0);
+          const uint64_t off = (uint64_t)(((kk >> 2) * C::SUB_BYTES + (kk & 3) * 32) >> 4);
+          mma_bf16_ss(tmem + C::s_col(X), dq + off, dk + off, IDESC_S, kk > 0);
         }
         mma_commit(&s_full[X]);
       };
       auto issue_pv = [&](int X, uint32_t g, int j) {
-        const uint32_t sV = smem_u32(smem + C::OFF_V + kv_slot(X, g) * C::T_BYTES);
+        const uint64_t dv = desc_sw128(smem_u32(smem + C::OFF_V + kv_slot(X, g) * C::T_BYTES), C::SUB_BYTES, 1024);
 #pragma unroll
         for (int kk = 0; kk < BKV / 16; ++kk)  // 16 keys = 8 TMEM columns of packed P; 2 atoms of V
-          mma_bf16_ts(tmem + C::o_col(X), tmem + C::s_col(X) + kk * 8,
-                      desc_sw128(sV + kk * 2048, C::SUB_BYTES, 1024), IDESC_O, (j | kk) != 0);
+          mma_bf16_ts(tmem + C::o_col(X), tmem + C::s_col(X) + kk * 8, dv + (uint64_t)(kk * (2048 >> 4)), IDESC_O,
+                      (j | kk) != 0);
         mma_commit(&pv_done[X]);
       };
       uint32_t gk = 0;          // K/V tiles consumed so far
@@ -393,17 +415,16 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
     // ---------------- softmax + output (warps 2..9) ----------------
     const int X = warp >= 6 ? 1 : 0;
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;  // query row in the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
     const uint32_t tS = tmem + lane_off + C::s_col(X);
     const uint32_t tO = tmem + lane_off + C::o_col(X);
+    uint8_t* box = smem + C::OFF_STG + (warp - 2) * 4096;
     const float sl2 = 1.4426950408889634f / sqrtf((float)HD);  // log2(e) / sqrt(hd)
     uint32_t gx = 0;  // tiles of this X processed so far (phases of s_full / p_full / pv_done)
     bool ok = true;
     for (int qb = qb0; qb < qb1 && ok; ++qb) {
       const int q0 = qb * 2 * BQ;
       if (X == 1 && !dual && !(q0 + BQ < p.Lq)) continue;  // this block has no tile B
-      const int qrow0 = c * p.Lq + q0;
       float m = -INFINITY, l = 0.0f;
       for (int j = 0; j < nt; ++j, ++gx) {
         if (!warp_wait(&s_full[X], gx & 1, &abort_flag, status)) { ok = false; break; }
@@ -466,27 +487,36 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
       if (!warp_wait(&pv_done[X], (gx - 1) & 1, &abort_flag, status)) { ok = false; break; }
       tc_fence_after();
       const float inv = 1.0f / l;
-      // tile B holds the next query rows, or (paired heads) the same rows of head hB
-      const int roff = dual ? 0 : X * BQ;
-      const bool row_ok = q0 + roff + r < p.Lq;
-      bf16* O = (bf16*)p.out + (long long)(qrow0 + roff + r) * p.ldo + (X ? hB : h) * HD;
+      // O / l as bf16, 64 columns at a time, through this warp's swizzled 32-row
+      // box and a TMA store: whole 128-byte row segments instead of one row per
+      // thread.  Rows at or past Lq fall outside the chunk in the output map and
+      // are not written.  Tile B holds the next query rows, or (paired heads)
+      // the same rows of head hB.
+      const int y0 = q0 + (dual ? 0 : X * BQ) + quad * 32;
+      const int x0 = (X ? hB : h) * HD;
 #pragma unroll 1
-      for (int i = 0; i < HD / 32; ++i) {
-        float t[32];
-        tmem_ld32(tO + i * 32, t);
-        if (row_ok) {
-          uint4* d4 = reinterpret_cast<uint4*>(O + i * 32);
+      for (int i = 0; i < HD / 64; ++i) {
+        float t[64];
+        tmem_ld32_nowait(tO + i * 64, *reinterpret_cast<float(*)[32]>(t));
+        tmem_ld32_nowait(tO + i * 64 + 32, *reinterpret_cast<float(*)[32]>(t + 32));
+        tmem_wait_ld();
+        uint32_t w[32];
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4)
-            d4[q4] = make_uint4(pack_bf16(t[q4 * 8] * inv, t[q4 * 8 + 1] * inv),
-                                pack_bf16(t[q4 * 8 + 2] * inv, t[q4 * 8 + 3] * inv),
-                                pack_bf16(t[q4 * 8 + 4] * inv, t[q4 * 8 + 5] * inv),
-                                pack_bf16(t[q4 * 8 + 6] * inv, t[q4 * 8 + 7] * inv));
+        for (int e = 0; e < 32; ++e) w[e] = pack_bf16(t[2 * e] * inv, t[2 * e + 1] * inv);
+        if (lane == 0) bulk_wait_read<0>();  // the previous store has read the box
+        __syncwarp();
+        stage_row(box, lane, w);
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&maps.o, x0 + 64 * i, y0, c, box);
+          bulk_commit();
         }
       }
       // the next block's PV overwrites O only after this thread's next P arrives
       tc_fence_before();
     }
+    if (lane == 0) bulk_wait_all();  // output stores have landed
   }
   tc_fence_before();
   __syncthreads();
@@ -494,6 +524,32 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
     tc_fence_after();
     tmem_dealloc(tmem, Cfg<HD>::TMEM_COLS);
   }
+}
+
+typedef CUresult (*EncodeTiledFn3)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The bf16 output as a 3-D tensor [n_chunks][Lq][cols] (row stride ld
+// elements), boxes of 32 rows x 64 columns of one chunk, 128-byte swizzle.
+bool make_out_map(CUtensorMap* map, void* base, int n_chunks, int Lq, long long cols, long long ld) {
+  static EncodeTiledFn3 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn3>(f);
+  });
+  if (!fn) return false;
+  cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)Lq, (cuuint64_t)n_chunks};
+  cuuint64_t strides[2] = {(cuuint64_t)ld * 2, (cuuint64_t)Lq * (cuuint64_t)ld * 2};
+  cuuint32_t box[3] = {64, 32, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int HD>
@@ -524,6 +580,7 @@ cudaError_t launch(const AttnParams& p, int* status, cudaStream_t s) {
     maps.kp = maps.k;
     maps.vp = maps.v;
   }
+  if (!make_out_map(&maps.o, p.out, p.n_chunks, p.Lq, w, p.ldo)) return cudaErrorInvalidValue;
   // query blocks of 256 per CTA: more when the key set is short (the setup of
   // a CTA, its Q loads and its O write-back are then amortised over more work)
   const long long keys = (long long)p.Lk * (1 + (p.pred_in_batch ? 1 : 0) + (p.succ_in_batch ? 1 : 0));
