@@ -18,35 +18,61 @@ __device__ __forceinline__ float gelu_erf(float x) {
 }
 __device__ __forceinline__ float silu(float x) { return x / (1.0f + expf(-x)); }
 
-// GELU x * Phi(x) with erf from Abramowitz and Stegun, Handbook of
-// Mathematical Functions, formula 7.1.26 (|error of erf| <= 1.5e-7):
-// erf(z) = 1 - (a1 t + a2 t^2 + a3 t^3 + a4 t^4 + a5 t^5) exp(-z^2),
-// t = 1 / (1 + p z), z >= 0; erf is odd.  Branch-free, used by the
-// tensor-core GEMM epilogue; the reciprocal and 2^x run on the MUFU unit
-// (approximate, relative error ~1e-7, well inside the formula's bound).
+// Reciprocal on the MUFU unit (approximate, relative error ~1e-7).
 __device__ __forceinline__ float rcp_approx(float x) {
   float y;
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-__device__ __forceinline__ float ex2_approx_f(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
 
-__device__ __forceinline__ float gelu_as(float x) {
-  const float z = fabsf(x) * 0.70710678118654752f;
-  const float t = rcp_approx(fmaf(0.3275911f, z, 1.0f));
-  float poly = fmaf(1.061405429f, t, -1.453152027f);
-  poly = fmaf(poly, t, 1.421413741f);
-  poly = fmaf(poly, t, -0.284496736f);
-  poly = fmaf(poly, t, 0.254829592f);
-  poly *= t;
-  const float e = ex2_approx_f(-z * z * 1.4426950408889634f);
-  const float erf_abs = fmaf(-poly, e, 1.0f);
-  const float erf_x = copysignf(erf_abs, x);
-  return 0.5f * x * (1.0f + erf_x);
+// GELU of two values, returned as a bf16 pair (low half = a), with erf from
+// Abramowitz and Stegun, Handbook of Mathematical Functions, formula 7.1.28
+// (|error of erf| <= 3e-7): erf(z) = 1 - 1 / (1 + a1 z + ... + a6 z^6)^16,
+// z >= 0; erf is odd.  Both lanes go through the packed fp32x2 instructions
+// of sm_100 (each lane rounded as the scalar instruction); the one
+// reciprocal per value runs on the MUFU unit, and there is no exponential.
+// For large z the 16th power overflows to +inf, whose reciprocal is 0:
+// erf = 1, the limit.  Used by the tensor-core GEMM's GELU epilogue.
+__device__ __forceinline__ uint64_t f32x2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f32x2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f32x2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t gelu2_bf16(float a, float b) {
+  constexpr uint64_t kAbs = 0x7FFFFFFF7FFFFFFFull, kSign = 0x8000000080000000ull;
+  const uint64_t x = f32x2_pack(a, b);
+  const uint64_t z = f32x2_mul(x & kAbs, f32x2_pack(0.70710678118654752f, 0.70710678118654752f));
+  uint64_t q = f32x2_fma(z, f32x2_pack(0.0000430638f, 0.0000430638f), f32x2_pack(0.0002765672f, 0.0002765672f));
+  q = f32x2_fma(q, z, f32x2_pack(0.0001520143f, 0.0001520143f));
+  q = f32x2_fma(q, z, f32x2_pack(0.0092705272f, 0.0092705272f));
+  q = f32x2_fma(q, z, f32x2_pack(0.0422820123f, 0.0422820123f));
+  q = f32x2_fma(q, z, f32x2_pack(0.0705230784f, 0.0705230784f));
+  q = f32x2_fma(q, z, f32x2_pack(1.0f, 1.0f));
+  q = f32x2_mul(q, q);  // ^2
+  q = f32x2_mul(q, q);  // ^4
+  q = f32x2_mul(q, q);  // ^8
+  q = f32x2_mul(q, q);  // ^16
+  float q0, q1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(q0), "=f"(q1) : "l"(q));
+  // |erf| = 1 - 1/q; with the sign of x, Phi = (1 + erf) / 2 = 0.5 + 0.5 erf
+  const uint64_t r = f32x2_pack(rcp_approx(q0), rcp_approx(q1));
+  const uint64_t e = f32x2_fma(r, f32x2_pack(-1.0f, -1.0f), f32x2_pack(1.0f, 1.0f));
+  const uint64_t es = (e & kAbs) | (x & kSign);
+  const uint64_t phi = f32x2_fma(es, f32x2_pack(0.5f, 0.5f), f32x2_pack(0.5f, 0.5f));
+  float g0, g1;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(g0), "=f"(g1) : "l"(f32x2_mul(x, phi)));
+  __nv_bfloat162 v = __floats2bfloat162_rn(g0, g1);
+  return *reinterpret_cast<uint32_t*>(&v);
 }
 
 // Ring offset of (row, col) of the head output: row = token of batch chunk,

@@ -351,13 +351,14 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
           tmem_ld32(tbase + g * 64, *reinterpret_cast<float(*)[32]>(v0));
           tmem_ld32(tbase + g * 64 + 32, *reinterpret_cast<float(*)[32]>(v0 + 32));
           add_bias<64>(e, col0, N, v);
+          uint32_t w[32];
           if (e.mode == EPI_GELU) {
 #pragma unroll
-            for (int i = 0; i < 64; ++i) v[i] = gelu_as(v[i]);
-          }
-          uint32_t w[32];
+            for (int i = 0; i < 32; ++i) w[i] = gelu2_bf16(v[2 * i], v[2 * i + 1]);
+          } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) w[i] = pack_bf16(v[2 * i], v[2 * i + 1]);
+            for (int i = 0; i < 32; ++i) w[i] = pack_bf16(v[2 * i], v[2 * i + 1]);
+          }
           if (e.cache && row < M && row >= e.cache_row0 && row < e.cache_row0 + e.cache_rows &&
               col0 >= e.cache_col0) {
             uint4* d = reinterpret_cast<uint4*>((bf16*)e.cache + (long long)(row - e.cache_row0) * e.ldc +
