@@ -263,6 +263,17 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
     uint8_t* box = smem + STG_OFF + (warp - 2) * 4096;
     const bool bf16_out = (e.mode == EPI_STORE && !e.out_f32) || e.mode == EPI_GELU;
     const bool reduce = e.mode == EPI_RESID || e.mode == EPI_RESID_GATED;
+    // hands accumulator buffer `b` back to the MMA warp once this warp's TMEM
+    // loads of it are complete
+    auto release_acc = [&](int b) {
+      tc_fence_before();
+      if (PAIR) {
+        __syncwarp();  // every lane's accumulator loads are complete
+        if (lane == 0) mbar_arrive_cluster(cluster_addr(&tempty_bar[b], 0));
+      } else {
+        mbar_arrive(&tempty_bar[b]);
+      }
+    };
     int it = 0;
     for (int t = unit0; t < num_tiles; t += units, ++it) {
       const int buf = it & 1;
@@ -275,6 +286,7 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
       const int row_base = m0 + quad * 32;
       const int row = row_base + lane;
       const uint32_t tbase = tmem_base + ((uint32_t)(quad * 32) << 16) + buf * BN + half * HALF;
+      bool released = false;  // accumulator buffer handed back to the MMA warp
       if (half * HALF >= BN) {
         // no columns for this warp group
       } else if (e.rope && n0 < 2 * e.rope_d) {
@@ -342,14 +354,8 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
           }
         }
       } else if (bf16_out) {
-#pragma unroll 1
-        for (int g = 0; g < HALF / 64; ++g) {
-          const int col0 = n0 + g * 64;
-          if (col0 >= N) break;  // uniform
-          float v[64];
-          float* v0 = v;
-          tmem_ld32(tbase + g * 64, *reinterpret_cast<float(*)[32]>(v0));
-          tmem_ld32(tbase + g * 64 + 32, *reinterpret_cast<float(*)[32]>(v0 + 32));
+        // bias (+ GELU), bf16, optional cache copy, one TMA store of 64 columns
+        auto convert_store = [&](int col0, float (&v)[64]) {
           add_bias<64>(e, col0, N, v);
           uint32_t w[32];
           if (e.mode == EPI_GELU) {
@@ -375,6 +381,25 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
             tma_store_2d(&maps.out, col0, row_base, box);
             bulk_commit();
           }
+        };
+        // The accumulator goes back to the MMA warp as soon as this warp's
+        // last column group is in registers; that group's conversion and
+        // store run after the release (the GELU epilogue held the accumulator
+        // for most of a tile's MMA time).
+        float v[64];
+        tmem_ld32(tbase, *reinterpret_cast<float(*)[32]>(v));
+        tmem_ld32(tbase + 32, *reinterpret_cast<float(*)[32]>(v + 32));
+        if (HALF / 64 == 2 && n0 + 64 < N) {
+          convert_store(n0, v);
+          tmem_ld32(tbase + 64, *reinterpret_cast<float(*)[32]>(v));
+          tmem_ld32(tbase + 96, *reinterpret_cast<float(*)[32]>(v + 32));
+          release_acc(buf);
+          released = true;
+          convert_store(n0 + 64, v);
+        } else {
+          release_acc(buf);
+          released = true;
+          convert_store(n0, v);
         }
       } else if (e.mode == EPI_EULER) {
 #pragma unroll 1
@@ -434,13 +459,7 @@ gemm_tc_kernel(const __grid_constant__ GemmMaps maps, int M, int N, int K, EpiPa
           }
         }
       }
-      tc_fence_before();
-      if (PAIR) {
-        __syncwarp();  // every lane's accumulator loads are complete
-        if (lane == 0) mbar_arrive_cluster(cluster_addr(&tempty_bar[buf], 0));
-      } else {
-        mbar_arrive(&tempty_bar[buf]);
-      }
+      if (!released) release_acc(buf);
     }
     if (lane == 0) bulk_wait_all();  // stores and reductions have landed
   }
