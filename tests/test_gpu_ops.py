@@ -227,10 +227,13 @@ def test_self_attention_neighbour_buffers(dtype, hd, Lc, n, cached, succ, H):
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("Lq", [257, 700])
-def test_cross_attention_shared_keys(dtype, Lq):
+@pytest.mark.parametrize("hd,Lt", [(64, 64), (128, 77)])
+def test_cross_attention_shared_keys(dtype, Lq, hd, Lt):
     """Several 256-query blocks per CTA (short key set); Lq = 257 ends in a
-    one-tile block of 1 row, Lq = 700 in a block of two tiles (188 rows)."""
-    H, hd, n, Lt = 4, 64, 3, 64
+    one-tile block of 1 row, Lq = 700 in a block of two tiles (188 rows).
+    77 prompt keys leave most of the one key tile masked; the output rows of a
+    chunk's last block that fall past Lq must not land in the next chunk."""
+    H, n = 4, 3
     d = H * hd
     tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
     q = gen((n * Lq, d), 1.0, tdt, seed=32)
