@@ -585,7 +585,7 @@ cudaError_t launch(const AttnParams& p, int* status, cudaStream_t s) {
   // a CTA, its Q loads and its O write-back are then amortised over more work)
   const long long keys = (long long)p.Lk * (1 + (p.pred_in_batch ? 1 : 0) + (p.succ_in_batch ? 1 : 0));
   AttnParams q = p;
-  q.qblocks_per_cta = p.qblocks_per_cta > 0 ? p.qblocks_per_cta : (keys <= 1024 ? 4 : 1);
+  q.qblocks_per_cta = p.qblocks_per_cta > 0 ? p.qblocks_per_cta : (keys <= 1024 ? 5 : 1);
   const int nqb = (p.Lq + 2 * BQ - 1) / (2 * BQ);
   // A last block of one tile (Lq mod 256 in 1..128) costs a full block's
   // time for at most half its rows: pair the heads' last blocks in one column.
