@@ -225,6 +225,25 @@ def test_self_attention_neighbour_buffers(dtype, hd, Lc, n, cached, succ, H):
     assert rel_l2(f64(out), ref) < (1e-2 if dtype == "bf16" else 1e-5)
 
 
+@pytest.mark.parametrize("hd", [64, 128])
+@pytest.mark.parametrize("Lc", [5, 20])
+def test_attention_chunks_shorter_than_an_output_box(hd, Lc):
+    """Chunks of fewer query rows than the 32-row output box of the
+    tensor-core path: self-attention with a cached predecessor, and
+    cross-attention to a short prompt."""
+    H, n = 2, 3
+    d = H * hd
+    qkv = gen((n * Lc, 3 * d), 1.0, torch.bfloat16, seed=34)
+    q, k, v = qkv[:, :d], qkv[:, d:2 * d], qkv[:, 2 * d:]
+    cache = gen((Lc, 2 * d), 1.0, torch.bfloat16, seed=35)
+    out = run_attn(q, k, v, n, Lc, H, hd, Lc, Lc, 1, cache[:, :d], cache[:, d:])
+    ref = oracle_self_attention(f64(q), f64(k), f64(v), n, Lc, H, f64(cache[:, :d]), f64(cache[:, d:]))
+    assert rel_l2(f64(out), ref) < 1e-2
+    kv = gen((9, 2 * d), 1.0, torch.bfloat16, seed=36)
+    out = run_attn(q, kv[:, :d], kv[:, d:], n, Lc, H, hd, 9, 0, 0)
+    assert rel_l2(f64(out), dit.attention(f64(q), f64(kv[:, :d]), f64(kv[:, d:]), H)) < 1e-2
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("Lq", [257, 700])
 @pytest.mark.parametrize("hd,Lt", [(64, 64), (128, 77)])
