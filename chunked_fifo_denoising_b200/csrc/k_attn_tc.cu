@@ -16,8 +16,9 @@
 // block holds one tile of rows (3120 = 12 x 256 + 48) has the last blocks of
 // heads h and h + 1 paired in one CTA as its tiles A and B, each with its own
 // head's K/V.  10 warps:
-//   warp 0      TMA producer: Q_A, Q_B once; K and V tiles of 128 keys into two
-//               2-stage rings, each tile from whichever buffer it belongs to
+//   warp 0      TMA producer: Q_A, Q_B per block; K and V tiles of 128 keys
+//               into two 2-stage rings, each tile from whichever buffer it
+//               belongs to
 //   warp 1      TMEM owner + MMA issuer, tiles ping-ponged on the tensor core:
 //               S_X = Q_X K_j^T (M=128, N=128, K=hd) into TMEM, then
 //               O_X += P_X V_j with P_X read from TMEM (the TS form)
@@ -25,7 +26,8 @@
 //               row: S row from TMEM, online max/sum in the log2 domain, P as
 //               bf16 written back over S in TMEM; O is rescaled in TMEM only when
 //               a row maximum grows by more than 2^8 (exact: the final division
-//               uses the same reference)
+//               uses the same reference); O / l leaves through a swizzled 4 KB
+//               box per warp and TMA stores that clip at the end of the chunk
 // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+hd) O_B [256+hd,256+2hd).
 // Every mbarrier wait is bounded.
 #include <mutex>
