@@ -216,6 +216,16 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnParams p, int* status)
     tmem_alloc(&tmem_base_sh, C::TMEM_COLS);
     tmem_relinquish();
   }
+  if (warp == 0 && lane == 0) {  // tensor-map descriptors into the cache before the first copies
+    prefetch_tmap(&maps.q);
+    prefetch_tmap(&maps.k);
+    prefetch_tmap(&maps.v);
+    prefetch_tmap(&maps.o);
+    if (c == 0) {
+      prefetch_tmap(&maps.kp);
+      prefetch_tmap(&maps.vp);
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
